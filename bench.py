@@ -1,0 +1,386 @@
+"""Benchmark of the block-FP8 linear hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input
+on the headline layer (M=512 tokens, K=5120, N=25600, the largest linear of a
+32B-class decoder):
+  quantize_weight (BF16 W -> E4M3 codes + scales), dequantize (-> BF16),
+  linear_w8a16 (x BF16 . dequant(W)^T) and linear_w8a8 (x quantized per
+  1x128 K-group, then the FP8 GEMM).
+`value` = FLOPs of the step's two linears (2 * 2MNK) / device time of the
+step, summed over ranks / max over ranks. Per-call times, TFLOP/s, weight
+GB/s and roofline fractions are reported beside it. L2 is flushed between
+steps (a 512 MiB memset outside the step's CUDA events).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Multi-GPU (torchrun): replicas only -- each rank runs its own copy of the
+layer; there is no data-path collective (NCCL is used only for the barrier
+and the max-over-ranks timing reduction).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "block-FP8 linear TFLOP/s and weight-stream GB/s (M=512,K=5120,N=25600)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
+FLUSH_BYTES = 512 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="fp8blk", choices=["fp8blk", "reference"])
+    ap.add_argument("--workload", default="linear_m512_k5120_n25600")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        loaded = [r for r in rows if r[2] > 250.0] or rows
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(1, 5) if r[3][i] == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# --------------------------------------------------------------- oracle arm
+def oracle_sample_step(wl, wb, xb, n_rows):
+    """The step on the first n_rows output rows (n_rows % 128 == 0): every
+    stage's work is proportional to N, so this is the step scaled by n_rows/N."""
+    import oracle
+    w_s = wb[:n_rows]
+    q, s = oracle.quantize_weight(w_s)
+    oracle.dequantize(q, s)
+    oracle.linear_w8a16(xb, q, s, n_rows, wl.K)
+    qx, sx = oracle.act_quant(xb)
+    oracle.linear_w8a8(qx, sx, q, s, n_rows, wl.K)
+    return 4.0 * wl.M * n_rows * wl.K
+
+
+def calibrate_oracle_rows(wl, wb, xb, seconds: float) -> int:
+    t = time.perf_counter()
+    oracle_sample_step(wl, wb, xb, 128)
+    t1 = time.perf_counter() - t
+    blocks = max(1, min(-(-wl.N // 128), int(seconds / max(t1, 1e-6))))
+    return 128 * blocks
+
+
+def run_oracle(wl, wb, xb, seconds: float):
+    import oracle
+    rows = calibrate_oracle_rows(wl, wb, xb, seconds)
+    t = time.perf_counter()
+    flops = oracle_sample_step(wl, wb, xb, rows)
+    dt = time.perf_counter() - t
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"the step on {rows} of {wl.N} output rows (all M={wl.M} tokens, "
+                      f"K={wl.K}): {dt:.1f} s of CPU work"}
+
+
+def reference_arm(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from block_scaled_fp8_fp8blk_b200 import synth
+    wb = synth.bf16_bits(wl.weight_bf16())
+    xb = synth.bf16_bits(wl.x_bf16())
+    per_step = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    rows = calibrate_oracle_rows(wl, wb, xb, per_step)
+    for _ in range(args.warmup):
+        oracle_sample_step(wl, wb, xb, rows)
+    times = []
+    flops = 0.0
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        flops = oracle_sample_step(wl, wb, xb, rows)
+        times.append(time.perf_counter() - t)
+    total = sum(times)
+    value = flops * args.steps / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N,
+                   "sample_rows": rows, "parallelism": "single process, CPU threads"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: the step on {rows} of {wl.N} output rows"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def traffic_for(kernel_file: str, key: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    source is unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(key)
+        src = os.path.join(ROOT, "block_scaled_fp8_fp8blk_b200", "csrc", kernel_file)
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if rec and rec.get("source_sha256_16") == digest:
+            return rec.get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+def main():
+    args = parse()
+    from block_scaled_fp8_fp8blk_b200 import workloads
+    wl = workloads.ALL[args.workload]
+    if args.impl == "reference":
+        return reference_arm(args, wl)
+
+    import torch
+    import torch.distributed as dist
+
+    import block_scaled_fp8_fp8blk_b200 as fb
+    from block_scaled_fp8_fp8blk_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    M, K, N = wl.M, wl.K, wl.N
+    # replicas: each rank its own seeded copy of the layer
+    from dataclasses import replace
+    wl_r = replace(wl, seed=wl.seed + rank)
+    w_h = wl_r.weight_bf16()
+    x_h = wl_r.x_bf16()
+    w = w_h.to(dev)
+    x = x_h.to(dev)
+    ldq = -(-K // 16) * 16
+    q = torch.empty((N, ldq), dtype=torch.uint8, device=dev)[:, :K]
+    s = torch.empty((-(-N // 128), -(-K // 128)), dtype=torch.float32, device=dev)
+    wd = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    y16 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    y8 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws16 = torch.empty(max(1, fb.workspace_size(0, M, N, K)), dtype=torch.uint8, device=dev)
+    ws8 = torch.empty(max(1, fb.workspace_size(1, M, N, K)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev: ev[0].record()
+        fb.quantize_weight(w, q=q, scale_inv=s)
+        if ev: ev[1].record()
+        fb.dequantize(q, s, out=wd)
+        if ev: ev[2].record()
+        fb.linear_w8a16(x, q, s, out=y16, workspace=ws16)
+        if ev: ev[3].record()
+        fb.linear_w8a8(x, q, s, out=y8, workspace=ws8)
+        if ev: ev[4].record()
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert fb.read_device_error() == 0
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(visible.split(",")[local] if visible else str(local))
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.15)
+    for i in range(args.steps):
+        flush.zero_()
+        step(events[i])
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+
+    calls = ["quantize_weight", "dequantize", "linear_w8a16", "linear_w8a8"]
+    per_call = {c: [ev[j].elapsed_time(ev[j + 1]) for ev in events] for j, c in enumerate(calls)}
+    step_ms_total = sum(ev[0].elapsed_time(ev[4]) for ev in events)
+    t_local = torch.tensor([step_ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    step_ms_max = float(t_local.item()) / args.steps
+
+    flops_step = 2.0 * (2.0 * M * N * K)
+    value = world * flops_step / (step_ms_max * 1e-3) / 1e12
+
+    peaks, peak_kind = load_peaks()
+    NB, KB = -(-N // 128), -(-K // 128)
+    wbytes = N * K + 4 * NB * KB
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    call_stats = {}
+    for c in calls:
+        ms = statistics.mean(per_call[c])
+        if c == "quantize_weight":
+            alg = 2 * N * K + N * K + 4 * NB * KB
+            ach = alg / (ms * 1e-3) / 1e9
+            call_stats[c] = {"us": 1e3 * ms, "bound": "hbm", "achieved": ach, "unit": "GB/s",
+                             "peak": peaks["hbm_gbs"], "frac": ach / peaks["hbm_gbs"],
+                             "alg_bytes": alg}
+        elif c == "dequantize":
+            alg = N * K + 4 * NB * KB + 2 * N * K
+            ach = alg / (ms * 1e-3) / 1e9
+            call_stats[c] = {"us": 1e3 * ms, "bound": "hbm", "achieved": ach, "unit": "GB/s",
+                             "peak": peaks["hbm_gbs"], "frac": ach / peaks["hbm_gbs"],
+                             "alg_bytes": alg}
+        else:
+            fl = 2.0 * M * N * K
+            tf = fl / (ms * 1e-3) / 1e12
+            peak = peaks["bf16_tflops"] if c == "linear_w8a16" else fp8_peak
+            hbm_bytes = wbytes + 2 * M * K + 2 * M * N
+            call_stats[c] = {"us": 1e3 * ms, "bound": "tensor", "achieved": tf, "unit": "TFLOP/s",
+                             "peak": peak, "frac": tf / peak, "alg_flops": fl,
+                             "weight_stream_gbs": wbytes / (ms * 1e-3) / 1e9,
+                             "hbm_frac": hbm_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    dominant = max(calls, key=lambda c: call_stats[c]["us"])
+    d = call_stats[dominant]
+    kernel_file = {"quantize_weight": "quant.cu", "dequantize": "quant.cu",
+                   "linear_w8a16": "gemm_w8a16.cu", "linear_w8a8": "gemm_w8a8.cu"}[dominant]
+    roofline = {"kernel": dominant, "bound": d["bound"], "achieved": d["achieved"],
+                "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
+                "peak_kind": f"{peak_kind} burst" + (" x2 (fp8 nominal ratio)" if dominant == "linear_w8a8" else ""),
+                "traffic": traffic_for(kernel_file, f"{dominant}:{wl.name}")}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3/bf16 operands, f32 accumulate", "data": "synthetic",
+        "config": {"workload": wl.name, "M": M, "K": K, "N": N,
+                   "step": "quantize_weight + dequantize + linear_w8a16 + linear_w8a8",
+                   "l2": "flushed between steps (512 MiB memset outside the step events)",
+                   "parallelism": f"replicas x{world}"},
+        "weight_stream_gbs": {c: call_stats[c]["weight_stream_gbs"]
+                              for c in ("linear_w8a16", "linear_w8a8")},
+        "calls": call_stats, "roofline": roofline,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk,
+    }
+
+    # e2e: the same step through the public API with inputs from pinned host
+    # memory and the two linear outputs read back, every step.
+    if not args.no_e2e:
+        w_pin = w_h.pin_memory()
+        x_pin = x_h.pin_memory()
+        y16_pin = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        y8_pin = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        e_steps = max(3, min(args.steps, 20))
+        for _ in range(2):
+            w.copy_(w_pin, non_blocking=True); x.copy_(x_pin, non_blocking=True)
+            step()
+            y16_pin.copy_(y16, non_blocking=True); y8_pin.copy_(y8, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e_steps):
+            w.copy_(w_pin, non_blocking=True); x.copy_(x_pin, non_blocking=True)
+            step()
+            y16_pin.copy_(y16, non_blocking=True); y8_pin.copy_(y8, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1) / e_steps], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        line["e2e"] = {"value": world * flops_step / (float(te.item()) * 1e-3) / 1e12,
+                       "unit": "TFLOP/s", "ms_per_step": float(te.item()), "steps": e_steps,
+                       "h2d_bytes_per_step": 2 * N * K + 2 * M * K,
+                       "d2h_bytes_per_step": 2 * 2 * M * N}
+    else:
+        line["e2e"] = None
+
+    assert fb.read_device_error() == 0
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = run_oracle(wl, synth.bf16_bits(w_h), synth.bf16_bits(x_h), 12.0)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

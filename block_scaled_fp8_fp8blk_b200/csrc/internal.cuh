@@ -1,0 +1,47 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fp8blk {
+
+struct Launch {
+  cudaStream_t stream;
+  unsigned* err;  // device error word (bounded-wait time-outs)
+  int num_sms;
+};
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return cdiv(a, b) * b; }
+
+cudaError_t launch_quantize_weight(const Launch& L, const uint16_t* w, int64_t N, int64_t K,
+                                   int64_t ldw, uint8_t* q, int64_t ldq, float* scale_inv);
+cudaError_t launch_dequantize(const Launch& L, const uint8_t* q, int64_t ldq,
+                              const float* scale_inv, int64_t N, int64_t K, uint16_t* w,
+                              int64_t ldw);
+cudaError_t launch_quantize_act(const Launch& L, const uint16_t* x, int64_t M, int64_t K,
+                                int64_t ldx, uint8_t* qx, int64_t ldqx, float* sx, int64_t ldsx);
+cudaError_t launch_encode_e4m3(const Launch& L, const float* v, int64_t n, uint8_t* codes);
+
+cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, const float* sx,
+                             int64_t ldsx, const uint8_t* q, int64_t ldq, const float* scale_inv,
+                             uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K);
+
+size_t w8a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
+                              int64_t ldq, const float* scale_inv, uint16_t* y, int64_t ldy,
+                              int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes);
+
+// 2-D tiled tensor map with 128-byte swizzling over a row-major matrix
+// [outer][inner] whose rows are row_bytes apart; out-of-bounds reads are
+// zero-filled. Returns false when the driver rejects the description.
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+
+// Sets the kernel's dynamic shared-memory limit once per device.
+cudaError_t ensure_smem_limit(const void* kernel, size_t bytes);
+
+}  // namespace fp8blk

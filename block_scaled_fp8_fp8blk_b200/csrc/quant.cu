@@ -1,0 +1,234 @@
+// Elementwise stages of the block-FP8 linear: the weight converter, the
+// dequantizer, the 1 x 128 activation quantizer and the bare E4M3 codec.
+// All are HBM-bound streams: 16-byte vector loads and stores, one pass over
+// the data (the converter keeps its 128 x 128 block in registers between the
+// amax reduction and the encoding).
+#include "internal.cuh"
+#include "ptx.cuh"
+
+namespace fp8blk {
+namespace {
+
+// Per-halfword |bf16| maximum. For non-NaN values the magnitude order equals
+// the unsigned order of (bits & 0x7FFF), so integer maxima give the exact amax.
+__device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t w) {
+  return __vmaxu2(acc, w & 0x7FFF7FFFu);
+}
+
+__device__ __forceinline__ uint32_t absmax_u4(uint32_t acc, const uint4& v) {
+  acc = absmax2(acc, v.x);
+  acc = absmax2(acc, v.y);
+  acc = absmax2(acc, v.z);
+  return absmax2(acc, v.w);
+}
+
+// Four BF16 values (two words, element 0 in the low half of w01) divided by
+// d (IEEE division, round to nearest even) and encoded to E4M3 with
+// saturation; code i lands in byte i.
+__device__ __forceinline__ uint32_t encode4(uint32_t w01, uint32_t w23, float d) {
+  const float q0 = __fdiv_rn(bf16_lo_to_f32(w01), d);
+  const float q1 = __fdiv_rn(bf16_hi_to_f32(w01), d);
+  const float q2 = __fdiv_rn(bf16_lo_to_f32(w23), d);
+  const float q3 = __fdiv_rn(bf16_hi_to_f32(w23), d);
+  return cvt_e4m3x2(q1, q0) | (cvt_e4m3x2(q3, q2) << 16);
+}
+
+__device__ __forceinline__ uint2 encode8(const uint4& v, float d) {
+  return make_uint2(encode4(v.x, v.y, d), encode4(v.z, v.w, d));
+}
+
+// Loads 8 BF16 values at p (16-byte aligned); elements at or past `valid`
+// read as +0, which never changes an amax.
+__device__ __forceinline__ uint4 load8_bf16(const uint16_t* p, int valid) {
+  if (valid >= 8) return __ldcs(reinterpret_cast<const uint4*>(p));
+  uint32_t e[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) e[t] = (t < valid) ? static_cast<uint32_t>(p[t]) : 0u;
+  return make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16),
+                    e[6] | (e[7] << 16));
+}
+
+__device__ __forceinline__ void store8_codes(uint8_t* p, uint2 c, int valid) {
+  if (valid >= 8) {
+    __stcs(reinterpret_cast<uint2*>(p), c);
+    return;
+  }
+#pragma unroll
+  for (int t = 0; t < 8; ++t)
+    if (t < valid) p[t] = static_cast<uint8_t>(((t < 4 ? c.x : c.y) >> (8 * (t & 3))) & 0xFFu);
+}
+
+// ------------------------------------------------------------- converter
+// One CTA per 128 x 128 block (FastVideo PR #1829, "Changes", converter
+// bullet): 256 threads x 8 chunks of 8 BF16 values stay in registers; the
+// block amax is reduced across the CTA; every element is then divided by
+// s = amax / 448 and encoded.
+__global__ void __launch_bounds__(256) quantize_weight_kernel(
+    const uint16_t* __restrict__ w, int64_t N, int64_t K, int64_t ldw, uint8_t* __restrict__ q,
+    int64_t ldq, float* __restrict__ scale_inv, int KB) {
+  const int64_t blk = blockIdx.x;
+  const int64_t nb = blk / KB, kb = blk - nb * KB;
+  const int64_t n0 = nb * 128, k0 = kb * 128;
+  const int rows = static_cast<int>((N - n0 < 128 ? N - n0 : 128));
+  const int cols = static_cast<int>((K - k0 < 128 ? K - k0 : 128));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  uint4 v[8];
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = tid + 256 * i;
+    const int r = c >> 4, kk = (c & 15) * 8;
+    v[i] = make_uint4(0, 0, 0, 0);
+    if (r < rows && kk < cols) v[i] = load8_bf16(w + (n0 + r) * ldw + k0 + kk, cols - kk);
+    m2 = absmax_u4(m2, v[i]);
+  }
+  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t red[8];
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  m = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) m = max(m, red[i]);
+
+  const float amax = __uint_as_float(m << 16);
+  const float s = __fdiv_rn(amax, 448.0f);
+  if (tid == 0) scale_inv[blk] = s;
+  // An all-zero block has s = 0: its +-0 elements keep their sign under a
+  // division by 1 instead.
+  const float d = (amax == 0.0f) ? 1.0f : s;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = tid + 256 * i;
+    const int r = c >> 4, kk = (c & 15) * 8;
+    if (r < rows && kk < cols) store8_codes(q + (n0 + r) * ldq + k0 + kk, encode8(v[i], d), cols - kk);
+  }
+}
+
+// ----------------------------------------------------------- dequantizer
+// w[n][k] = BF16(float(E4M3(q[n][k])) * s[n/128][k/128]): one warp per row at
+// a time, 16 codes (one 16-byte load, two 16-byte stores) per lane-step.
+__device__ __forceinline__ uint32_t dequant2(uint32_t codes16, float s) {
+  const uint32_t h2 = e4m3x2_to_f16x2(codes16);
+  return cvt_bf16x2(__fmul_rn(f16_hi_to_f32(h2), s), __fmul_rn(f16_lo_to_f32(h2), s));
+}
+
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ q, int64_t ldq,
+                                                         const float* __restrict__ scale_inv,
+                                                         int64_t N, int64_t K, int KB,
+                                                         uint16_t* __restrict__ w, int64_t ldw) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * 8;
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); n < N; n += warps) {
+    const uint8_t* qrow = q + n * ldq;
+    uint16_t* wrow = w + n * ldw;
+    const float* srow = scale_inv + (n >> 7) * KB;
+    for (int64_t k = static_cast<int64_t>(lane) * 16; k < K; k += 32 * 16) {
+      const float s = __ldg(srow + (k >> 7));
+      if (k + 16 <= K) {
+        const uint4 c = __ldcs(reinterpret_cast<const uint4*>(qrow + k));
+        const uint4 o0 = make_uint4(dequant2(c.x, s), dequant2(c.x >> 16, s), dequant2(c.y, s),
+                                    dequant2(c.y >> 16, s));
+        const uint4 o1 = make_uint4(dequant2(c.z, s), dequant2(c.z >> 16, s), dequant2(c.w, s),
+                                    dequant2(c.w >> 16, s));
+        __stcs(reinterpret_cast<uint4*>(wrow + k), o0);
+        __stcs(reinterpret_cast<uint4*>(wrow + k + 8), o1);
+      } else {
+        for (int64_t t = k; t < K; ++t)
+          wrow[t] = static_cast<uint16_t>(dequant2(qrow[t], s) & 0xFFFFu);
+      }
+    }
+  }
+}
+
+// -------------------------------------------------- activation quantizer
+// 1 x 128 K-groups: a half-warp per group (16 lanes x 8 BF16), amax by
+// shuffles, s = amax / 448, codes = E4M3(x / s). Each warp walks one row at a
+// time with its two half-warps on alternating groups; the loop trip count is
+// uniform across the warp so the shuffles always see all 32 lanes.
+__global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x,
+                                                           int64_t M, int64_t K, int64_t ldx,
+                                                           uint8_t* __restrict__ qx, int64_t ldqx,
+                                                           float* __restrict__ sx, int64_t ldsx,
+                                                           int KB) {
+  const int lane = threadIdx.x & 31, half = lane >> 4, j = lane & 15;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * 8;
+  const int pairs = (KB + 1) / 2;
+  for (int64_t m = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); m < M; m += warps) {
+    const uint16_t* xrow = x + m * ldx;
+    for (int p = 0; p < pairs; ++p) {
+      const int kb = 2 * p + half;
+      const int64_t k = static_cast<int64_t>(kb) * 128 + 8 * j;
+      const bool valid = kb < KB && k < K;
+      const int nvalid = valid ? static_cast<int>((K - k < 8 ? K - k : 8)) : 0;
+      const uint4 v = valid ? load8_bf16(xrow + k, nvalid) : make_uint4(0, 0, 0, 0);
+      uint32_t m2 = absmax_u4(0u, v);
+      uint32_t mx = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+      const float amax = __uint_as_float(mx << 16);
+      const float s = __fdiv_rn(amax, 448.0f);
+      const float d = (amax == 0.0f) ? 1.0f : s;
+      if (valid) store8_codes(qx + m * ldqx + k, encode8(v, d), nvalid);
+      if (kb < KB && j == 0) sx[static_cast<int64_t>(kb) * ldsx + m] = s;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ codec
+__global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ v, int64_t n,
+                                                     uint8_t* __restrict__ out) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x * 4;
+  for (int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4; i < n;
+       i += stride) {
+    if (i + 4 <= n) {
+      const float4 f = __ldcs(reinterpret_cast<const float4*>(v + i));
+      const uint32_t c = cvt_e4m3x2(f.y, f.x) | (cvt_e4m3x2(f.w, f.z) << 16);
+      __stcs(reinterpret_cast<unsigned int*>(out + i), c);
+    } else {
+      for (int64_t t = i; t < n; ++t) out[t] = static_cast<uint8_t>(cvt_e4m3x2(0.0f, v[t]) & 0xFFu);
+    }
+  }
+}
+
+int grid_for_rows(int64_t rows, int num_sms) {
+  const int64_t ctas = cdiv(rows, 8);
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  return static_cast<int>(ctas < cap ? ctas : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_weight(const Launch& L, const uint16_t* w, int64_t N, int64_t K,
+                                   int64_t ldw, uint8_t* q, int64_t ldq, float* scale_inv) {
+  const int64_t NB = cdiv(N, 128), KB = cdiv(K, 128);
+  if (NB * KB > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  quantize_weight_kernel<<<static_cast<unsigned>(NB * KB), 256, 0, L.stream>>>(
+      w, N, K, ldw, q, ldq, scale_inv, static_cast<int>(KB));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const Launch& L, const uint8_t* q, int64_t ldq,
+                              const float* scale_inv, int64_t N, int64_t K, uint16_t* w,
+                              int64_t ldw) {
+  dequantize_kernel<<<grid_for_rows(N, L.num_sms), 256, 0, L.stream>>>(
+      q, ldq, scale_inv, N, K, static_cast<int>(cdiv(K, 128)), w, ldw);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_act(const Launch& L, const uint16_t* x, int64_t M, int64_t K,
+                                int64_t ldx, uint8_t* qx, int64_t ldqx, float* sx, int64_t ldsx) {
+  quantize_act_kernel<<<grid_for_rows(M, L.num_sms), 256, 0, L.stream>>>(
+      x, M, K, ldx, qx, ldqx, sx, ldsx, static_cast<int>(cdiv(K, 128)));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode_e4m3(const Launch& L, const float* v, int64_t n, uint8_t* codes) {
+  const int64_t ctas = cdiv(n, 1024);
+  const int64_t cap = static_cast<int64_t>(L.num_sms) * 16;
+  encode_kernel<<<static_cast<unsigned>(ctas < cap ? ctas : cap), 256, 0, L.stream>>>(v, n, codes);
+  return cudaGetLastError();
+}
+
+}  // namespace fp8blk

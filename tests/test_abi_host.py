@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/fp8blk.h declares, and rejects bad arguments before it
+makes any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_scaled_fp8_fp8blk_b200 as fb
+from block_scaled_fp8_fp8blk_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8blk.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fbuild.build_cuda()
+    return fb.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FP8BLK_EXPORT\s+[\w\s\*]+?\b(fp8blk_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_symbols()
+    for n in ("fp8blk_quantize_weight", "fp8blk_dequantize", "fp8blk_linear_w8a16",
+              "fp8blk_linear_w8a8"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(fb.EXPORTS)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.fp8blk_version() == 100
+    for code in range(7):
+        assert lib.fp8blk_status_string(code)
+    assert lib.fp8blk_status_string(99) == b"unknown status"
+
+
+def test_workspace_size(lib):
+    M, N, K = 77, 1000, 1000
+    ldqx, ldsx, KB = 1008, 128, 8
+    sx_off = -(-M * ldqx // 256) * 256
+    assert lib.fp8blk_workspace_size(1, M, N, K) == sx_off + KB * ldsx * 4
+    assert lib.fp8blk_workspace_size(0, 0, N, K) == 0
+    assert lib.fp8blk_workspace_size(1, M, N, 0) == 0
+    assert lib.fp8blk_workspace_size(2, M, N, K) == 0
+    assert lib.fp8blk_workspace_size(1, -1, N, K) == 0
+
+
+# Arguments below are rejected before any CUDA call, so they run without a GPU.
+P = 1 << 20          # a 16-byte-aligned fake address (never dereferenced)
+PM = P + 2           # misaligned
+
+
+def test_quantize_weight_validation(lib):
+    f = lib.fp8blk_quantize_weight
+    assert f(P, -1, 128, 128, P, 128, P, None) == 1
+    assert f(P, 0, 128, 128, P, 128, P, None) == 0          # empty: nothing to do
+    assert f(P, 128, 0, 128, P, 128, P, None) == 0
+    assert f(None, 128, 128, 128, P, 128, P, None) == 1
+    assert f(P, 128, 128, 64, P, 128, P, None) == 1         # ldw < K
+    assert f(P, 128, 128, 128, P, 100, P, None) == 1        # ldq < K
+    assert f(P, 128, 128, 132, P, 128, P, None) == 2        # ldw % 8
+    assert f(P, 128, 128, 128, P, 136, P, None) == 2        # ldq % 16
+    assert f(PM, 128, 128, 128, P, 128, P, None) == 2
+    assert f(P, 128, 128, 128, P, 128, P + 1, None) == 2    # scale pointer 4-byte
+
+
+def test_dequantize_validation(lib):
+    f = lib.fp8blk_dequantize
+    assert f(P, 128, P, -5, 128, P, 128, None) == 1
+    assert f(P, 128, P, 0, 128, P, 128, None) == 0
+    assert f(P, 120, P, 128, 128, P, 128, None) == 1
+    assert f(P, 144, P, 128, 128, P, 132, None) == 2
+    assert f(PM, 128, P, 128, 128, P, 128, None) == 2
+
+
+def test_quantize_act_validation(lib):
+    f = lib.fp8blk_quantize_act
+    assert f(P, 64, 256, 256, P, 256, P, 32, None) == 1     # ldsx < M
+    assert f(P, 64, 256, 256, P, 256, P, 66, None) == 2     # ldsx % 4
+    assert f(P, 64, 256, 256, P, 256, PM, 64, None) == 2
+    assert f(P, 0, 256, 256, P, 256, P, 64, None) == 0
+
+
+@pytest.mark.parametrize("name", ["fp8blk_linear_w8a16", "fp8blk_linear_w8a8"])
+def test_linear_validation(lib, name):
+    f = getattr(lib, name)
+    M, N, K = 64, 384, 256
+    ws = lib.fp8blk_workspace_size(1 if name.endswith("a8") else 0, M, N, K)
+    ok = (P, K, P, K, P, P, N, M, N, K, P if ws else None, ws, None)
+
+    def call(**kw):
+        a = list(ok)
+        idx = dict(x=0, ldx=1, q=2, ldq=3, s=4, y=5, ldy=6, M=7, N=8, K=9, ws=10, wsb=11)
+        for k, v in kw.items():
+            a[idx[k]] = v
+        return f(*a)
+
+    assert call(M=-1) == 1
+    assert call(M=0) == 0 and call(N=0) == 0
+    assert call(x=None) == 1 and call(q=None) == 1 and call(s=None) == 1 and call(y=None) == 1
+    assert call(ldx=K - 8) == 1 and call(ldq=K - 16) == 1 and call(ldy=N - 8) == 1
+    assert call(ldx=K + 4) == 2 and call(ldq=K + 8) == 2 and call(ldy=N + 4) == 2
+    assert call(x=PM) == 2 and call(q=PM) == 2 and call(y=PM) == 2 and call(s=P + 2) == 2
+    if ws:
+        assert call(ws=None) == 4
+        assert call(wsb=ws - 1) == 4
+        assert call(ws=P + 16) == 4   # workspace must be 256-byte aligned
+
+
+def test_encode_validation(lib):
+    f = lib.fp8blk_encode_e4m3
+    assert f(P, -1, P, None) == 1
+    assert f(P, 0, P, None) == 0
+    assert f(PM, 16, P, None) == 2
+    assert f(None, 16, P, None) == 1
+
+
+def test_read_error_rejects_null(lib):
+    assert lib.fp8blk_read_device_error(None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(fb, "_lib", None)
+    monkeypatch.setattr(fb, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        fb.lib()

@@ -1,0 +1,256 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bit-exact: the E4M3 codec (every float32 bit pattern), the converter, the
+dequantizer and the activation quantizer. Within tolerance (relative Frobenius
+2e-3, per element 2^-7 |ref| + 1e-2 rms(ref)): both linears, on every
+workload shape, full outputs for the small ones and seeded row samples at
+full size. Plus edge cases: empty sizes, K = 0, ragged tiles, padded leading
+dimensions with canaries, one-hot rows."""
+import numpy as np
+import pytest
+import torch
+
+import block_scaled_fp8_fp8blk_b200 as fb
+import oracle
+from block_scaled_fp8_fp8blk_b200 import synth, workloads as W
+from helpers import bf16_bits, bf16_to_f64, check_linear
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def device():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    major, _ = torch.cuda.get_device_capability(0)
+    assert major == 10, "the library targets compute capability 10.x"
+    torch.cuda.set_device(0)
+    fb.lib()
+    yield
+    assert fb.read_device_error() == 0, "a kernel reported a timed-out wait"
+
+
+def to_dev_bf16(bits: np.ndarray, ld: int | None = None):
+    R, C = bits.shape
+    ld = ld or C
+    buf = torch.zeros((R, ld), dtype=torch.int16)
+    buf[:, :C] = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return buf.view(torch.bfloat16).to(DEV)[:, :C]
+
+
+def to_dev_u8(a: np.ndarray, ld: int | None = None):
+    R, C = a.shape
+    ld = ld or -(-C // 16) * 16
+    buf = torch.zeros((R, ld), dtype=torch.uint8)
+    buf[:, :C] = torch.from_numpy(np.ascontiguousarray(a))
+    return buf.to(DEV)[:, :C]
+
+
+def u8(t) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+_W_CACHE = {}
+
+
+def weight_case(wl):
+    """(W bits, oracle q, oracle s) for a workload's weight, cached."""
+    key = (wl.N, wl.K, wl.row_gain_sigma, wl.seed)
+    if key not in _W_CACHE:
+        _W_CACHE.clear()
+        wb = synth.bf16_bits(wl.weight_bf16())
+        q, s = oracle.quantize_weight(wb)
+        _W_CACHE[key] = (wb, q, s)
+    return _W_CACHE[key]
+
+
+# ------------------------------------------------------------------ codec
+def test_encode_every_float32():
+    n = 1 << 28
+    for lo in range(0, 1 << 32, n):
+        v = torch.arange(n, dtype=torch.int64, device=DEV) + lo
+        v = torch.where(v >= (1 << 31), v - (1 << 32), v).to(torch.int32).view(torch.float32)
+        codes = u8(fb.encode_e4m3(v))
+        del v
+        assert oracle.count_code_mismatches(lo, codes) == 0, hex(lo)
+
+
+# -------------------------------------------------------------- converter
+CONVERTER_CASES = [W.TINY, W.RAGGED, W.Workload("one", 1, 1, 1), W.Workload("odd", 3, 200, 129),
+                   W.Workload("full128", 1, 256, 256, row_gain_sigma=1.0), W.QKV, W.LINEAR_512]
+
+
+@pytest.mark.parametrize("wl", CONVERTER_CASES, ids=lambda w: w.name)
+def test_quantize_weight_bit_exact(wl):
+    wb, q_ref, s_ref = weight_case(wl)
+    ldw = -(-wl.K // 8) * 8 + (8 if wl is W.RAGGED else 0)
+    ldq = -(-wl.K // 16) * 16 + (16 if wl in (W.RAGGED, W.TINY) else 0)
+    w_d = to_dev_bf16(wb, ldw)
+    qbuf = torch.full((wl.N, ldq), 0xA5, dtype=torch.uint8, device=DEV)
+    s_d = torch.full((-(-wl.N // 128), -(-wl.K // 128)), -1.0, device=DEV)
+    fb.quantize_weight(w_d, q=qbuf[:, :wl.K], scale_inv=s_d)
+    qh = u8(qbuf)
+    assert np.array_equal(qh[:, :wl.K], q_ref)
+    assert np.all(qh[:, wl.K:] == 0xA5), "wrote past K"
+    assert np.array_equal(s_d.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+def test_quantize_zero_blocks_and_signs():
+    N, K = 260, 300
+    w = np.zeros((N, K), np.float32)
+    w[0, 0] = -0.0
+    w[:128, 128:256] = -0.0
+    w[200, 299] = 3.0
+    w[200, 298] = -1e-30
+    w[5, 200] = 2.0 ** -130          # a BF16 subnormal block amax
+    w[6, 201] = -2.0 ** -133
+    wb = synth.bf16_bits(synth.to_bf16(w))
+    q_ref, s_ref = oracle.quantize_weight(wb)
+    q_d, s_d = fb.quantize_weight(to_dev_bf16(wb))
+    assert np.array_equal(u8(q_d), q_ref)
+    assert np.array_equal(s_d.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+def test_quantize_every_bf16_value():
+    allb = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = (allb.astype(np.uint32) << 16).view(np.float32)
+    v = allb[np.isfinite(vals)]
+    n = -(-v.size // 128) * 128
+    wb = np.zeros(n, np.uint16)
+    wb[:v.size] = v
+    wb = wb.reshape(-1, 128)
+    q_ref, s_ref = oracle.quantize_weight(wb)
+    q_d, s_d = fb.quantize_weight(to_dev_bf16(wb))
+    assert np.array_equal(u8(q_d), q_ref)
+    assert np.array_equal(s_d.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+# ------------------------------------------------------------ dequantizer
+@pytest.mark.parametrize("wl", [W.TINY, W.RAGGED, W.Workload("odd", 3, 200, 129), W.LINEAR_512],
+                         ids=lambda w: w.name)
+def test_dequantize_bit_exact(wl):
+    wb, q, s = weight_case(wl)
+    ref = oracle.dequantize(q, s)
+    ldw = -(-wl.K // 8) * 8 + 8
+    out = torch.full((wl.N, ldw), 0x7FC1, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+    fb.dequantize(to_dev_u8(q), torch.from_numpy(s).to(DEV), out=out[:, :wl.K])
+    got = bf16_bits(out)
+    assert np.array_equal(got[:, :wl.K], ref)
+    assert np.all(got[:, wl.K:] == 0x7FC1)
+
+
+def test_dequantize_all_codes_many_scales():
+    rng = np.random.default_rng(7)
+    codes = np.tile(np.arange(256, dtype=np.uint8), (256, 2))   # [256, 512]
+    codes[(codes == 0x7F) | (codes == 0xFF)] = 0x00
+    s = (rng.random((2, 4)) * 10.0 ** rng.integers(-30, 3, (2, 4))).astype(np.float32)
+    s[0, 0] = 0.0
+    s[1, 3] = 1.0
+    ref = oracle.dequantize(codes, s)
+    got = bf16_bits(fb.dequantize(to_dev_u8(codes), torch.from_numpy(s).to(DEV)))
+    assert np.array_equal(got, ref)
+
+
+# --------------------------------------------------- activation quantizer
+@pytest.mark.parametrize("wl", [W.TINY, W.RAGGED, W.Workload("k130", 5, 130, 8), W.LINEAR_512,
+                                W.LARGE_4096], ids=lambda w: w.name)
+def test_quantize_act_bit_exact(wl):
+    xb = synth.bf16_bits(wl.x_bf16())
+    qx_ref, sx_ref = oracle.act_quant(xb)
+    qx_d, sx_d = fb.quantize_act(to_dev_bf16(xb, -(-wl.K // 8) * 8 + 8))
+    assert np.array_equal(u8(qx_d), qx_ref)
+    sx = sx_d.cpu().numpy()[:, :wl.M].T       # group-major -> [M][KB]
+    assert np.array_equal(sx.view(np.uint32), sx_ref.view(np.uint32))
+
+
+# ---------------------------------------------------------------- linears
+LINEAR_FULL = [W.TINY, W.RAGGED, W.Workload("k130_n300", 50, 130, 300),
+               W.Workload("m200_k384_n640", 200, 384, 640, row_gain_sigma=0.5)]
+LINEAR_SAMPLED = [W.QKV, W.O_PROJ, W.GATE_UP, W.DOWN, W.LINEAR_512, W.LARGE_4096, W.LARGE_16384]
+SMALL_M = [w.with_m(m) for w in W.DECODER_SHAPES for m in W.SMALL_M]
+
+
+def run_linear(wl, mode, rows=None, ldx_pad=0, ldy_pad=0):
+    wb, q_ref, s_ref = weight_case(wl)
+    xb = synth.bf16_bits(wl.x_bf16())
+    q_d, s_d = fb.quantize_weight(to_dev_bf16(wb))
+    assert np.array_equal(u8(q_d), q_ref)
+    x_d = to_dev_bf16(xb, -(-wl.K // 8) * 8 + ldx_pad)
+    ldy = -(-wl.N // 8) * 8 + ldy_pad
+    ybuf = torch.full((wl.M, ldy), 0x7FC1, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+    f = fb.linear_w8a16 if mode == "w8a16" else fb.linear_w8a8
+    f(x_d, q_d, s_d, out=ybuf[:, :wl.N])
+    torch.cuda.synchronize()
+    ybits = bf16_bits(ybuf)
+    assert np.all(ybits[:, wl.N:] == 0x7FC1), "wrote past N"
+    if mode == "w8a16":
+        ref = oracle.linear_w8a16(xb, q_ref, s_ref, wl.N, wl.K, rows=rows)
+    else:
+        qx, sx = oracle.act_quant(xb)
+        ref = oracle.linear_w8a8(qx, sx, q_ref, s_ref, wl.N, wl.K, rows=rows)
+    y = bf16_to_f64(ybuf[:, :wl.N])
+    if rows is not None:
+        y = y[rows]
+    return check_linear(y, ref, f"{wl.name}/{mode}")
+
+
+@pytest.mark.parametrize("mode", ["w8a16", "w8a8"])
+@pytest.mark.parametrize("wl", LINEAR_FULL, ids=lambda w: w.name)
+def test_linear_full_output(wl, mode):
+    run_linear(wl, mode, ldx_pad=8, ldy_pad=8)
+
+
+@pytest.mark.parametrize("mode", ["w8a16", "w8a8"])
+@pytest.mark.parametrize("wl", SMALL_M, ids=lambda w: w.name)
+def test_linear_small_m(wl, mode):
+    run_linear(wl, mode, rows=wl.checked_rows(64))
+
+
+@pytest.mark.parametrize("mode", ["w8a16", "w8a8"])
+@pytest.mark.parametrize("wl", LINEAR_SAMPLED, ids=lambda w: w.name)
+def test_linear_full_size_sampled_rows(wl, mode):
+    count = 256 if wl.M > 512 else 64
+    run_linear(wl, mode, rows=wl.checked_rows(count))
+
+
+@pytest.mark.parametrize("mode", ["w8a16", "w8a8"])
+def test_linear_empty_and_k0(mode):
+    f = fb.linear_w8a16 if mode == "w8a16" else fb.linear_w8a8
+    q = torch.zeros((16, 0), dtype=torch.uint8, device=DEV)
+    s = torch.zeros((1, 1), dtype=torch.float32, device=DEV)
+    x = torch.zeros((8, 0), dtype=torch.bfloat16, device=DEV)
+    y = torch.full((8, 16), 1.0, dtype=torch.bfloat16, device=DEV)
+    f(x, q, s, out=y)
+    assert torch.all(y == 0)
+    x2 = torch.zeros((0, 64), dtype=torch.bfloat16, device=DEV)
+    q2 = torch.zeros((16, 64), dtype=torch.uint8, device=DEV)
+    y2 = f(x2, q2, s)
+    assert y2.shape == (0, 16)
+
+
+def test_w8a16_one_hot_rows_reproduce_dequantized_weight():
+    # x = e_k gives P = the exact BF16 image of the code, acc = fl(code * s),
+    # y = BF16(acc) -- the dequantizer's value, bit for bit.
+    wl = W.RAGGED
+    wb, q, s = weight_case(wl)
+    ks = np.array([0, 1, 127, 128, 500, 999])
+    x = np.zeros((ks.size, wl.K), np.float32)
+    x[np.arange(ks.size), ks] = 1.0
+    y = fb.linear_w8a16(to_dev_bf16(synth.bf16_bits(synth.to_bf16(x))), to_dev_u8(q),
+                        torch.from_numpy(s).to(DEV))
+    deq = oracle.dequantize(q, s)
+    got = bf16_bits(y)
+    for i, k in enumerate(ks):
+        assert np.array_equal(got[i], deq[:, k])
+
+
+def test_repeat_calls_are_deterministic():
+    wl = W.Workload("m300_k640_n512", 300, 640, 512)
+    wb, q, s = weight_case(wl)
+    x_d = to_dev_bf16(synth.bf16_bits(wl.x_bf16()))
+    q_d, s_d = to_dev_u8(q), torch.from_numpy(s).to(DEV)
+    for f in (fb.linear_w8a16, fb.linear_w8a8):
+        a = bf16_bits(f(x_d, q_d, s_d))
+        b = bf16_bits(f(x_d, q_d, s_d))
+        assert np.array_equal(a, b)
