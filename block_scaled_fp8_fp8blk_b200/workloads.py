@@ -2,8 +2,9 @@
 
 Shapes follow the decoder of the pages' 32B-class text encoder (hidden 5120,
 fused QKV 8192 + 1024 + 1024, o_proj 8192 -> 5120, MLP 25600); the largest
-linear, 25600 x 5120, is the one whose BF16 copy is the "~0.26 GB" temporary
-of the Hopper route (FastVideo PR #1829, "Checklist").
+linear, 25600 x 5120, matches the size of the BF16 temporary that the Hopper
+route materializes per call, about a quarter of a gigabyte (FastVideo PR
+#1829, "Checklist").
 """
 from __future__ import annotations
 

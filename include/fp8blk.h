@@ -60,8 +60,8 @@ typedef void* fp8blk_stream;
 
 /* ---------------------------------------------------------------------------
  * (1) Converter: BF16 weight -> E4M3 codes + weight_scale_inv.
- * FastVideo PR #1829, section "Changes", converter bullet ("E4M3 weight plus
- * [N/128, K/128] weight_scale_inv"). For each 128 x 128 block:
+ * FastVideo PR #1829, section "Changes", converter bullet (E4M3 codes with a
+ * float weight_scale_inv grid of shape [N/128, K/128]). For each 128 x 128 block:
  *   amax = max |W| over the block's in-bounds elements (ragged edge blocks
  *          are not padded with anything but zeros),
  *   s    = amax / 448            (float division, round to nearest even),
@@ -115,8 +115,8 @@ FP8BLK_EXPORT fp8blk_status fp8blk_quantize_act(const void* x, int64_t M, int64_
  * (3) Linear, BF16 activations x block-FP8 weight ("W8A16"):
  *   y[m][n] = BF16( sum_kb s[n/128][kb] * P_kb[m][n] ),
  *   P_kb[m][n] = sum_{k in slab kb} x[m][k] * E4M3(q[n][k])   (FP32)
- * i.e. y = x . dequant(W)^T (FastVideo PR #1829, "Purpose": "the arithmetic
- * the FlashInfer path performs internally"), with the block scale applied to
+ * i.e. y = x . dequant(W)^T (FastVideo PR #1829, "Purpose": the same
+ * computation as the Blackwell groupwise GEMM), with the block scale applied to
  * the FP32 partial of each 128-wide K slab and FP32 accumulation across
  * slabs. Tensor cores see the exact BF16 image of each E4M3 code.
  *   x : BF16 [M][ldx], ldx >= K, ldx % 8 == 0                        (input)

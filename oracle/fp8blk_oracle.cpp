@@ -11,12 +11,11 @@
 //   * section "Changes", converter bullet: weights are E4M3 codes plus one
 //     float weight_scale_inv per 128x128 block, grid [N/128, K/128];
 //   * section "Purpose": each linear multiplies the activations by the
-//     dequantized weight, "the arithmetic the FlashInfer path performs
-//     internally";
+//     dequantized weight, which the page states is the same computation the
+//     Blackwell groupwise GEMM carries out inside;
 //   * section "Changes", tests bullet: the dequantizer equals the scale
 //     broadcast over its block times the code.
-// Steps the page leaves open are read as follows (each also listed in the
-// design notes): scale_inv = amax / 448 in float; a code is E4M3(W / s) with
+// Steps the page leaves open are read as follows: scale_inv = amax / 448 in float; a code is E4M3(W / s) with
 // a float division, round-to-nearest-even and saturation to +-448; an
 // all-zero block gets s = 0 and sign-preserving zero codes; the scale grid is
 // ceil-divided and amax covers in-bounds elements only; activations use
@@ -237,8 +236,8 @@ int64_t orc_count_code_mismatches(uint64_t lo, int64_t n, const uint8_t* codes, 
 }
 
 // ----------------------------------------------------- (a1) weight converter
-// FastVideo PR #1829, "Changes", converter bullet: E4M3 weight plus a float
-// weight_scale_inv [N/128, K/128]. w is BF16 [N][ldw]; q is [N][ldq];
+// FastVideo PR #1829, "Changes", converter bullet: the checkpoint holds the
+// E4M3 codes and a float weight_scale_inv grid of shape [N/128, K/128]. w is BF16 [N][ldw]; q is [N][ldq];
 // scale_inv is dense [ceil(N/128)][ceil(K/128)].
 void orc_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q,
                          int64_t ldq, float* scale_inv, int nthreads) {
@@ -272,7 +271,8 @@ void orc_dequantize(const uint8_t* q, int64_t ldq, const float* scale_inv, int64
 
 // --------------------------------------------------- (a3) activation quantize
 // The Blackwell route quantizes activations before the groupwise GEMM
-// (FastVideo PR #1829, "Changes", loader bullet: "the Triton quantizer").
+// (FastVideo PR #1829, "Changes", loader bullet, which names a Triton
+// activation quantizer for the Blackwell runtime).
 // Groups are 1 x 128 along K with the weight recipe. sx is [M][ceil(K/128)].
 void orc_act_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* qx,
                    int64_t ldqx, float* sx, int nthreads) {

@@ -33,7 +33,7 @@ def device():
 
 def to_dev_bf16(bits: np.ndarray, ld: int | None = None):
     R, C = bits.shape
-    ld = ld or C
+    ld = ld or -(-C // 8) * 8
     buf = torch.zeros((R, ld), dtype=torch.int16)
     buf[:, :C] = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
     return buf.view(torch.bfloat16).to(DEV)[:, :C]

@@ -1,7 +1,7 @@
 """Pins of the oracle's converter, dequantizer, activation quantizer and the two
 FP64 linears against independent routes: a hand-worked example, torch's
-float32 division / float8 cast / bfloat16 cast ("the reference broadcast" of
-FastVideo PR #1829, section "Changes", tests bullet), numpy float64 matmul on
+float32 division / float8 cast / bfloat16 cast (the scale broadcast over each
+block that FastVideo PR #1829, section "Changes", tests bullet, checks against), numpy float64 matmul on
 small shapes, closed forms (one-hot rows, constant blocks, zero blocks) and
 the format's invariants (the largest code of a block is 448)."""
 import numpy as np
@@ -96,8 +96,8 @@ def test_block_max_code_is_448(wl, weights):
 
 
 def test_roundtrip_within_e4m3_precision(wl, weights):
-    # FastVideo PR #1829, "Changes", tests bullet: the FP8 round trip stays
-    # within E4M3 precision: relative 2^-4 for normals, absolute 2^-10 * s for
+    # FastVideo PR #1829, "Changes", tests bullet: the FP8 round trip is held
+    # to the precision of E4M3: relative 2^-4 for normals, absolute 2^-10 * s for
     # subnormals, plus the final BF16 rounding (2^-9 relative).
     wb, q, s = weights
     wf = f32_from_bf16(wb).astype(np.float64)
