@@ -39,6 +39,7 @@ EXPORTS = {
     "fp8blk_quantize_act": (_st, [_p, _i64, _i64, _i64, _p, _i64, _p, _i64, _p]),
     "fp8blk_linear_w8a16": (_st, [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]),
     "fp8blk_linear_w8a8": (_st, [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]),
+    "fp8blk_linear_w8a8_noalloc": (_st, [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p]),
     "fp8blk_workspace_size": (_sz, [_int, _i64, _i64, _i64]),
     "fp8blk_encode_e4m3": (_st, [_p, _i64, _p, _p]),
     "fp8blk_read_device_error": (_st, [ctypes.POINTER(ctypes.c_uint32)]),

@@ -126,6 +126,10 @@ cudaError_t ensure_smem_limit(const void* kernel, size_t bytes) {
   return e;
 }
 
+// The launch context of the current device (stream, error word, SM count),
+// for entry points defined in other files.
+fp8blk_status current_launch(fp8blk_stream stream, Launch* L) { return make_launch(stream, L); }
+
 }  // namespace fp8blk
 
 using namespace fp8blk;

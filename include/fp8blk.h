@@ -151,6 +151,34 @@ FP8BLK_EXPORT fp8blk_status fp8blk_linear_w8a8(const void* x, int64_t ldx, const
                                  void* workspace, size_t workspace_bytes,
                                  fp8blk_stream stream);
 
+/* ---------------------------------------------------------------------------
+ * W8A8 linear without a workspace argument. (The pages have no counterpart:
+ * this is a calling convenience of this library.) For callers that cannot
+ * allocate device memory -- e.g. a runtime that plans every buffer before it
+ * starts serving and forbids allocation afterwards, or host code that must
+ * not call cudaMalloc because it can synchronize the device and stall other
+ * streams. Computes exactly what fp8blk_linear_w8a8 computes, with the same
+ * arguments minus the workspace; its scratch is a fixed array of
+ * FP8BLK_NOALLOC_SCRATCH_BYTES built into the library, present on every GPU
+ * that loads it until the process exits. The call itself allocates nothing.
+ *  - Limit: the problem must satisfy fp8blk_workspace_size(1, M, N, K) <=
+ *    FP8BLK_NOALLOC_SCRATCH_BYTES (M * round_up(K, 16) bytes of codes plus the
+ *    scales; e.g. M = 2048 at K = 5120); larger problems return
+ *    FP8BLK_ERR_WORKSPACE before anything is launched.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address once; make that first call before any stream
+ *    capture.
+ *  - All calls share the one array: calls that can overlap on the GPU (on
+ *    different streams, or from different threads) race on it and must be
+ *    ordered by the caller.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED_DEVICE, WORKSPACE (too large), CUDA.
+ * ------------------------------------------------------------------------- */
+#define FP8BLK_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+FP8BLK_EXPORT fp8blk_status fp8blk_linear_w8a8_noalloc(const void* x, int64_t ldx, const uint8_t* q,
+                                                       int64_t ldq, const float* scale_inv, void* y,
+                                                       int64_t ldy, int64_t M, int64_t N, int64_t K,
+                                                       fp8blk_stream stream);
+
 /* Workspace bytes for a linear: mode 0 = W8A16, 1 = W8A8. Pure host function;
  * returns 0 for an invalid mode or negative sizes. */
 FP8BLK_EXPORT size_t fp8blk_workspace_size(int mode, int64_t M, int64_t N, int64_t K);
