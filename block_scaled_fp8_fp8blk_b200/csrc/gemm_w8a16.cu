@@ -83,7 +83,8 @@ __global__ void __launch_bounds__(320, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(afull + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BT;
+  // Token tiles of one weight tile are adjacent in the grid (shared through L2).
+  const int m0 = blockIdx.x * BT, n0 = blockIdx.y * 128;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -131,29 +132,29 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // The x tile of a stage has landed once the expansion warps report the
+      // A buffer full (they waited on the stage's TMA barrier first), so the
+      // MMA thread waits only on afull and pempty. Descriptors are formed
+      // once; stepping through shared memory adds (bytes >> 4) to them.
+      const uint64_t xdesc0 = sw128_kmajor_desc(smem_addr(sX));
       int stage = 0, buf = 0, issued = 0;
-      uint32_t phase = 0, bphase = 0;
+      uint32_t bphase = 0;
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&afull[buf], bphase, err, kErrWaitMma)) break;
-        if (!mbar_wait(&full[stage], phase, err, kErrWaitMma)) break;
         if (!mbar_wait(&pempty[buf], bphase ^ 1u, err, kErrWaitMma)) break;
         tc_fence_after_sync();
-        const uint32_t xb = smem_addr(sX + stage * C::X_BYTES);
+        const uint64_t xd = xdesc0 + static_cast<uint64_t>((stage * C::X_BYTES) >> 4);
         const uint32_t d = tmem + static_cast<uint32_t>(C::TMEM_P + buf * BT);
         const uint32_t a = tmem + static_cast<uint32_t>(C::TMEM_A + buf * 64);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t bsa = xb + static_cast<uint32_t>((k >> 2) * C::X_ATOM + (k & 3) * 32);
-          mma_f16_ts(d, a + 8u * k, sw128_kmajor_desc(bsa), C::IDESC, k > 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < 8; ++k)
+          mma_f16_ts(d, a + 8u * k, xd + static_cast<uint64_t>(((k >> 2) * C::X_ATOM + (k & 3) * 32) >> 4),
+                     C::IDESC, k > 0 ? 1u : 0u);
         tc_commit(&empty[stage]);
         tc_commit(&aempty[buf]);
         tc_commit(&pfull[buf]);
         ++issued;
-        if (++stage == C::STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        if (++stage == C::STAGES) stage = 0;
         if (++buf == 2) {
           buf = 0;
           bphase ^= 1u;
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(320, 1)
     // -------------------------------------------------- promotion/epilogue
     const int quad = warp & 3;
     const int n = n0 + quad * 32 + lane;
-    const float* sw_row = sw + static_cast<int64_t>(blockIdx.x) * KB;
+    const float* sw_row = sw + static_cast<int64_t>(blockIdx.y) * KB;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::TMEM_P;
     float acc[BT];
 #pragma unroll
@@ -233,13 +234,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[i] = fmaf(__uint_as_float(p[i]), s, acc[i]);
       } else {
-#pragma unroll
-        for (int j = 0; j < BT / 32; ++j) {
-          uint32_t p[32];
-          tmem_ld32x32(t + 32u * j, p);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) acc[32 * j + i] = fmaf(__uint_as_float(p[i]), s, acc[32 * j + i]);
-        }
+        tmem_axpy<BT / 32>(t, s, acc);
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -282,7 +277,7 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
   auto kern = w8a16_gemm_kernel<BT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(cdiv(N, 128)), static_cast<unsigned>(cdiv(M, BT)));
+  dim3 grid(static_cast<unsigned>(cdiv(M, BT)), static_cast<unsigned>(cdiv(N, 128)));
   kern<<<grid, C::THREADS, C::SMEM, L.stream>>>(tq, tx, sw, reinterpret_cast<__nv_bfloat16*>(y),
                                                 ldy, static_cast<int>(M), static_cast<int>(N),
                                                 static_cast<int>(cdiv(K, 128)), L.err);
@@ -296,10 +291,10 @@ size_t w8a16_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
 cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                               int64_t ldq, const float* sw, uint16_t* y, int64_t ldy, int64_t M,
                               int64_t N, int64_t K, void*, size_t) {
+  if (cdiv(N, 128) > 65535) return cudaErrorInvalidValue;
   if (M <= 16) return launch_bt<16>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
   if (M <= 32) return launch_bt<32>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
   if (M <= 64) return launch_bt<64>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
-  if (cdiv(M, 128) > 65535) return cudaErrorInvalidValue;
   return launch_bt<128>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
 }
 

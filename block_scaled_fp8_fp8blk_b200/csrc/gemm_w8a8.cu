@@ -62,7 +62,9 @@ __global__ void __launch_bounds__(W8A8Cfg<BN>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * C::BM;
+  // Token tiles of one weight tile are adjacent in the grid, so they run
+  // together and read the weight tile from DRAM once.
+  const int m0 = blockIdx.x * C::BM, n0 = blockIdx.y * BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -108,19 +110,22 @@ __global__ void __launch_bounds__(W8A8Cfg<BN>::THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // Descriptors are formed once; stepping through shared memory adds
+      // (bytes >> 4) to their start-address field.
+      const uint64_t adesc0 = sw128_kmajor_desc(smem_addr(sA));
+      const uint64_t bdesc0 = sw128_kmajor_desc(smem_addr(sB));
       int stage = 0, buf = 0, issued = 0;
       uint32_t phase = 0, tphase = 0;
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&tempty[buf], tphase ^ 1u, err, kErrWaitMma)) break;
         if (!mbar_wait(&full[stage], phase, err, kErrWaitMma)) break;
         tc_fence_after_sync();
-        const uint32_t a0 = smem_addr(sA + stage * C::A_BYTES);
-        const uint32_t b0 = smem_addr(sB + stage * C::B_BYTES);
+        const uint64_t ad = adesc0 + static_cast<uint64_t>((stage * C::A_BYTES) >> 4);
+        const uint64_t bd = bdesc0 + static_cast<uint64_t>((stage * C::B_BYTES) >> 4);
         const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          mma_f8f6f4_ss(d, sw128_kmajor_desc(a0 + 32u * k), sw128_kmajor_desc(b0 + 32u * k),
-                        C::IDESC, k > 0 ? 1u : 0u);
+          mma_f8f6f4_ss(d, ad + 2u * k, bd + 2u * k, C::IDESC, k > 0 ? 1u : 0u);
         tc_commit(&empty[stage]);
         tc_commit(&tfull[buf]);
         ++issued;
@@ -167,14 +172,7 @@ __global__ void __launch_bounds__(W8A8Cfg<BN>::THREADS, 1)
         break;
       }
       tc_fence_after_sync();
-      const uint32_t t = t_row + static_cast<uint32_t>(buf * BN);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t r[32];
-        tmem_ld32x32(t + 32u * j, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[32 * j + i] = fmaf(__uint_as_float(r[i]), c, acc[32 * j + i]);
-      }
+      tmem_axpy<4>(t_row + static_cast<uint32_t>(buf * BN), c, acc);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -230,7 +228,7 @@ cudaError_t launch_bn(const Launch& L, const uint8_t* qx, int64_t ldqx, const fl
   auto kern = w8a8_gemm_kernel<BN>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(cdiv(N, BN)), static_cast<unsigned>(cdiv(M, 128)));
+  dim3 grid(static_cast<unsigned>(cdiv(M, 128)), static_cast<unsigned>(cdiv(N, BN)));
   kern<<<grid, C::THREADS, C::SMEM, L.stream>>>(ta, tb, sx, ldsx, sw,
                                                 reinterpret_cast<__nv_bfloat16*>(y), ldy,
                                                 static_cast<int>(M), static_cast<int>(N),
@@ -243,7 +241,7 @@ cudaError_t launch_bn(const Launch& L, const uint8_t* qx, int64_t ldqx, const fl
 cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, const float* sx,
                              int64_t ldsx, const uint8_t* q, int64_t ldq, const float* sw,
                              uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K) {
-  if (cdiv(M, 128) > 65535) return cudaErrorInvalidValue;
+  if (cdiv(N, 256) > 65535) return cudaErrorInvalidValue;
   return launch_bn<256>(L, qx, ldqx, sx, ldsx, q, ldq, sw, y, ldy, M, N, K);
 }
 

@@ -65,8 +65,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   const long long t0 = clock64();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 32; ++i) {
       if (mbar_try_wait(bar, parity)) return true;
+#ifdef FP8BLK_WAIT_BACKOFF_NS
+      __nanosleep(FP8BLK_WAIT_BACKOFF_NS);
+#endif
+    }
     if (clock64() - t0 > kWaitLimitCycles) {
       atomicOr(err, flag);
       return false;
@@ -252,6 +256,61 @@ __device__ __forceinline__ void tmem_ld32x16(uint32_t taddr, uint32_t (&r)[16]) 
       : "r"(taddr)
       : "memory");
   asm volatile("tcgen05.wait::ld.sync.aligned;" : FP8BLK_W8(r, 0), FP8BLK_W8(r, 8) : : "memory");
+}
+
+// Split form of the 32x32b.x32 load: issue, then wait carrying the
+// destination registers as in/out operands (no use can move above the wait).
+__device__ __forceinline__ void tmem_ld32x32_issue(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : FP8BLK_R8(r, 0), FP8BLK_R8(r, 8), FP8BLK_R8(r, 16), FP8BLK_R8(r, 24)
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : FP8BLK_W8(r, 0), FP8BLK_W8(r, 8), FP8BLK_W8(r, 16), FP8BLK_W8(r, 24)
+               :
+               : "memory");
+}
+
+// Empty volatile statement that claims to rewrite r: code reading r cannot
+// be scheduled above it (used to keep a load issued before the work that
+// should overlap it).
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
+  asm volatile("" : FP8BLK_W8(r, 0), FP8BLK_W8(r, 8), FP8BLK_W8(r, 16), FP8BLK_W8(r, 24));
+}
+
+// acc[j] += float(TMEM[lane, t + j]) * c for j < 32 * NCH: 32 columns per
+// load, the next load in flight while the current chunk is consumed.
+template <int NCH>
+__device__ __forceinline__ void tmem_axpy(uint32_t t, float c, float* acc) {
+  uint32_t pa[32], pb[32];
+  tmem_ld32x32_issue(t, pa);
+  tmem_ld_wait(pa);
+#pragma unroll
+  for (int j = 0; j < NCH; j += 2) {
+    if (j + 1 < NCH) {
+      tmem_ld32x32_issue(t + 32u * (j + 1), pb);
+      reg_fence(pa);
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[32 * j + i] = fmaf(__uint_as_float(pa[i]), c, acc[32 * j + i]);
+    if (j + 1 < NCH) {
+      tmem_ld_wait(pb);
+      if (j + 2 < NCH) {
+        tmem_ld32x32_issue(t + 32u * (j + 2), pa);
+        reg_fence(pb);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        acc[32 * (j + 1) + i] = fmaf(__uint_as_float(pb[i]), c, acc[32 * (j + 1) + i]);
+      if (j + 2 < NCH) tmem_ld_wait(pa);
+    }
+  }
 }
 
 // 32 lanes x 32 consecutive columns store (thread t writes lane base + t).

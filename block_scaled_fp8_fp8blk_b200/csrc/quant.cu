@@ -124,19 +124,33 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
     const uint8_t* qrow = q + n * ldq;
     uint16_t* wrow = w + n * ldw;
     const float* srow = scale_inv + (n >> 7) * KB;
-    for (int64_t k = static_cast<int64_t>(lane) * 16; k < K; k += 32 * 16) {
-      const float s = __ldg(srow + (k >> 7));
-      if (k + 16 <= K) {
-        const uint4 c = __ldcs(reinterpret_cast<const uint4*>(qrow + k));
-        const uint4 o0 = make_uint4(dequant2(c.x, s), dequant2(c.x >> 16, s), dequant2(c.y, s),
-                                    dequant2(c.y >> 16, s));
-        const uint4 o1 = make_uint4(dequant2(c.z, s), dequant2(c.z >> 16, s), dequant2(c.w, s),
-                                    dequant2(c.w >> 16, s));
-        __stcs(reinterpret_cast<uint4*>(wrow + k), o0);
-        __stcs(reinterpret_cast<uint4*>(wrow + k + 8), o1);
-      } else {
-        for (int64_t t = k; t < K; ++t)
-          wrow[t] = static_cast<uint16_t>(dequant2(qrow[t], s) & 0xFFFFu);
+    // Four 16-code chunks per lane per step: all four loads are issued before
+    // any conversion, so each warp keeps 2 KB of reads in flight.
+    for (int64_t base = 0; base < K; base += 4 * 32 * 16) {
+      uint4 c[4];
+      float s[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t k = base + u * 512 + lane * 16;
+        c[u] = make_uint4(0, 0, 0, 0);
+        s[u] = 0.0f;
+        if (k < K) s[u] = __ldg(srow + (k >> 7));
+        if (k + 16 <= K) c[u] = __ldcs(reinterpret_cast<const uint4*>(qrow + k));
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t k = base + u * 512 + lane * 16;
+        if (k + 16 <= K) {
+          const uint4 o0 = make_uint4(dequant2(c[u].x, s[u]), dequant2(c[u].x >> 16, s[u]),
+                                      dequant2(c[u].y, s[u]), dequant2(c[u].y >> 16, s[u]));
+          const uint4 o1 = make_uint4(dequant2(c[u].z, s[u]), dequant2(c[u].z >> 16, s[u]),
+                                      dequant2(c[u].w, s[u]), dequant2(c[u].w >> 16, s[u]));
+          __stcs(reinterpret_cast<uint4*>(wrow + k), o0);
+          __stcs(reinterpret_cast<uint4*>(wrow + k + 8), o1);
+        } else if (k < K) {
+          for (int64_t t = k; t < K; ++t)
+            wrow[t] = static_cast<uint16_t>(dequant2(qrow[t], s[u]) & 0xFFFFu);
+        }
       }
     }
   }
@@ -144,36 +158,32 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
 
 // -------------------------------------------------- activation quantizer
 // 1 x 128 K-groups: a half-warp per group (16 lanes x 8 BF16), amax by
-// shuffles, s = amax / 448, codes = E4M3(x / s). Each warp walks one row at a
-// time with its two half-warps on alternating groups; the loop trip count is
-// uniform across the warp so the shuffles always see all 32 lanes.
+// shuffles, s = amax / 448, codes = E4M3(x / s). Groups are numbered row-major
+// (g = m * KB + kb) and spread over the whole grid, 16 per CTA; lanes past
+// the last group still take part in the shuffles.
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x,
                                                            int64_t M, int64_t K, int64_t ldx,
                                                            uint8_t* __restrict__ qx, int64_t ldqx,
                                                            float* __restrict__ sx, int64_t ldsx,
                                                            int KB) {
-  const int lane = threadIdx.x & 31, half = lane >> 4, j = lane & 15;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * 8;
-  const int pairs = (KB + 1) / 2;
-  for (int64_t m = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); m < M; m += warps) {
-    const uint16_t* xrow = x + m * ldx;
-    for (int p = 0; p < pairs; ++p) {
-      const int kb = 2 * p + half;
-      const int64_t k = static_cast<int64_t>(kb) * 128 + 8 * j;
-      const bool valid = kb < KB && k < K;
-      const int nvalid = valid ? static_cast<int>((K - k < 8 ? K - k : 8)) : 0;
-      const uint4 v = valid ? load8_bf16(xrow + k, nvalid) : make_uint4(0, 0, 0, 0);
-      uint32_t m2 = absmax_u4(0u, v);
-      uint32_t mx = max(m2 & 0xFFFFu, m2 >> 16);
+  const int j = threadIdx.x & 15;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * 16 + (threadIdx.x >> 4);
+  const bool live = g < M * KB;
+  const int64_t m = live ? g / KB : 0;
+  const int kb = live ? static_cast<int>(g - m * KB) : 0;
+  const int64_t k = static_cast<int64_t>(kb) * 128 + 8 * j;
+  const bool valid = live && k < K;
+  const int nvalid = valid ? static_cast<int>((K - k < 8 ? K - k : 8)) : 0;
+  const uint4 v = valid ? load8_bf16(x + m * ldx + k, nvalid) : make_uint4(0, 0, 0, 0);
+  const uint32_t m2 = absmax_u4(0u, v);
+  uint32_t mx = max(m2 & 0xFFFFu, m2 >> 16);
 #pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-      const float amax = __uint_as_float(mx << 16);
-      const float s = __fdiv_rn(amax, 448.0f);
-      const float d = (amax == 0.0f) ? 1.0f : s;
-      if (valid) store8_codes(qx + m * ldqx + k, encode8(v, d), nvalid);
-      if (kb < KB && j == 0) sx[static_cast<int64_t>(kb) * ldsx + m] = s;
-    }
-  }
+  for (int off = 8; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+  const float amax = __uint_as_float(mx << 16);
+  const float s = __fdiv_rn(amax, 448.0f);
+  const float d = (amax == 0.0f) ? 1.0f : s;
+  if (valid) store8_codes(qx + m * ldqx + k, encode8(v, d), nvalid);
+  if (live && j == 0) sx[static_cast<int64_t>(kb) * ldsx + m] = s;
 }
 
 // ------------------------------------------------------------------ codec
@@ -219,7 +229,9 @@ cudaError_t launch_dequantize(const Launch& L, const uint8_t* q, int64_t ldq,
 
 cudaError_t launch_quantize_act(const Launch& L, const uint16_t* x, int64_t M, int64_t K,
                                 int64_t ldx, uint8_t* qx, int64_t ldqx, float* sx, int64_t ldsx) {
-  quantize_act_kernel<<<grid_for_rows(M, L.num_sms), 256, 0, L.stream>>>(
+  const int64_t ctas = cdiv(M * cdiv(K, 128), 16);
+  if (ctas > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  quantize_act_kernel<<<static_cast<unsigned>(ctas), 256, 0, L.stream>>>(
       x, M, K, ldx, qx, ldqx, sx, ldsx, static_cast<int>(cdiv(K, 128)));
   return cudaGetLastError();
 }
