@@ -156,9 +156,9 @@ __global__ void __launch_bounds__(W8A8Cfg<BN>::THREADS, 1)
     const float* sx_col = sx + m0 + row;  // sx[kb][m]: ldsx covers whole 128-row tiles
     const uint32_t t_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + col0;
 
-    float acc[128];
+    uint64_t acc[64];  // column pairs
 #pragma unroll
-    for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < 64; ++i) acc[i] = 0ull;
 
     int buf = 0;
     uint32_t tphase = 0;
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(W8A8Cfg<BN>::THREADS, 1)
         break;
       }
       tc_fence_after_sync();
-      tmem_axpy<4>(t_row + static_cast<uint32_t>(buf * BN), c, acc);
+      tmem_axpy2<4>(t_row + static_cast<uint32_t>(buf * BN), c, acc);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -190,10 +190,10 @@ __global__ void __launch_bounds__(W8A8Cfg<BN>::THREADS, 1)
       for (int j = 0; j < 16; ++j) {
         const int c = 8 * j;
         uint4 o;
-        o.x = cvt_bf16x2(acc[c + 1], acc[c + 0]);
-        o.y = cvt_bf16x2(acc[c + 3], acc[c + 2]);
-        o.z = cvt_bf16x2(acc[c + 5], acc[c + 4]);
-        o.w = cvt_bf16x2(acc[c + 7], acc[c + 6]);
+        o.x = cvt_bf16x2_pair(acc[c / 2 + 0]);
+        o.y = cvt_bf16x2_pair(acc[c / 2 + 1]);
+        o.z = cvt_bf16x2_pair(acc[c / 2 + 2]);
+        o.w = cvt_bf16x2_pair(acc[c / 2 + 3]);
         if (c + 8 <= ncols) {
           *reinterpret_cast<uint4*>(yrow + c) = o;
         } else if (c < ncols) {

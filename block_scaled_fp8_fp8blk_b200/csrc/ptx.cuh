@@ -328,6 +328,48 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------- registers and FP32x2
+// Warpgroup-wide register budget changes (all 128 threads of an aligned
+// warpgroup execute the same one). The per-warpgroup budgets of a kernel
+// must add up to no more than the registers it was launched with.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+// acc = p * c + acc on two FP32 lanes at once (each lane one rounded FMA).
+__device__ __forceinline__ void ffma2(uint64_t& acc, uint64_t p, uint64_t c) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(p), "l"(c));
+}
+
+// acc2[j] += (TMEM[lane, t + 2j], TMEM[lane, t + 2j + 1]) * (c, c) for
+// j < 16 * NCH, with packed FP32x2 FMAs (acc2 holds column pairs).
+template <int NCH>
+__device__ __forceinline__ void tmem_axpy2(uint32_t t, float c, uint64_t* acc2) {
+  const uint64_t c2 = pack_f32x2(c, c);
+#pragma unroll
+  for (int j = 0; j < NCH; ++j) {
+    uint32_t p[32];
+    tmem_ld32x32(t + 32u * j, p);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) ffma2(acc2[16 * j + i], pack_u32x2(p[2 * i], p[2 * i + 1]), c2);
+  }
+}
+
 // ------------------------------------------------------- FP8 conversions
 // Two floats -> two E4M3 codes, round to nearest even, saturating to +-448
 // (NaN -> 0x7F). `hi` lands in bits [8,16), `lo` in bits [0,8).
@@ -366,6 +408,13 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float hi, float lo) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// The two FP32 lanes of a pair -> bf16x2 (low lane -> low half), RNE.
+__device__ __forceinline__ uint32_t cvt_bf16x2_pair(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return cvt_bf16x2(hi, lo);
 }
 
 // Two E4M3 codes -> their exact BF16 images (bf16x2, low byte -> low half).
