@@ -69,18 +69,6 @@ __device__ __forceinline__ void expand16(const uint4& c, uint32_t* o) {
   o[7] = e4m3x2_to_bf16x2(c.w >> 16);
 }
 
-// Ring position bookkeeping: slot index and phase parity.
-struct Ring {
-  int slot = 0;
-  uint32_t phase = 0;
-  __device__ __forceinline__ void next(int depth) {
-    if (++slot == depth) {
-      slot = 0;
-      phase ^= 1u;
-    }
-  }
-};
-
 template <int BT, int NSUB>
 __global__ void __launch_bounds__(512, 1)
     w8a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_x,

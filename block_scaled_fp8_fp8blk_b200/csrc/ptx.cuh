@@ -87,6 +87,19 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, u
   return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
+// Position in a ring of mbarrier-guarded slots: slot index and the parity of
+// the phase that slot is on.
+struct Ring {
+  int slot = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next(int depth) {
+    if (++slot == depth) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 // Parity of the most recent phase of a ring slot that was used `uses` times.
 __device__ __forceinline__ uint32_t last_parity(int uses) { return static_cast<uint32_t>((uses - 1) & 1); }
 

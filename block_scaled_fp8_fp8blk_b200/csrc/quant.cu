@@ -22,19 +22,52 @@ __device__ __forceinline__ uint32_t absmax_u4(uint32_t acc, const uint4& v) {
   return absmax2(acc, v.w);
 }
 
-// Four BF16 values (two words, element 0 in the low half of w01) divided by
-// d (IEEE division, round to nearest even) and encoded to E4M3 with
-// saturation; code i lands in byte i.
-__device__ __forceinline__ uint32_t encode4(uint32_t w01, uint32_t w23, float d) {
-  const float q0 = __fdiv_rn(bf16_lo_to_f32(w01), d);
-  const float q1 = __fdiv_rn(bf16_hi_to_f32(w01), d);
-  const float q2 = __fdiv_rn(bf16_lo_to_f32(w23), d);
-  const float q3 = __fdiv_rn(bf16_hi_to_f32(w23), d);
-  return cvt_e4m3x2(q1, q0) | (cvt_e4m3x2(q3, q2) << 16);
+// The codes are E4M3(RN_f32(v / d)): the float quotient (IEEE division,
+// round to nearest even) rounded again to E4M3 with saturation.
+//
+// Division is the converter's costliest step, so when d >= 2^-125 a cheaper
+// route gives the same codes: with y = RN(1 / d), q = RN(v * y) lies within a
+// few float ulps of RN(v / d). E4M3 rounding can only tell them apart near one
+// of its decision points -- floats whose low 20 mantissa bits are 0x80000
+// (midpoints of the 3-bit mantissa grid) -- or in E4M3's subnormal range;
+// when any element of a warp's chunk is there (|low20 - 0x80000| <= 16 ulps,
+// or 0 < |q| < 2^-5) the whole chunk takes the exact quotient instead (a
+// warp-uniform branch; rare for real data). Checked exhaustively against the
+// exact quotient over every BF16 value v and every BF16 block maximum
+// (d = amax / 448).
+__device__ __forceinline__ bool near_e4m3_decision(float q) {
+  const uint32_t b = __float_as_uint(q) & 0x7FFFFFFFu;
+  return b != 0u && (b < 0x3D000000u || ((b & 0xFFFFFu) - 0x7FFF0u) <= 0x20u);
 }
 
+// Eight BF16 values -> eight E4M3 codes of RN_f32(v / d) (code i in byte i).
+// All 32 lanes of the warp must call this together.
 __device__ __forceinline__ uint2 encode8(const uint4& v, float d) {
-  return make_uint2(encode4(v.x, v.y, d), encode4(v.z, v.w, d));
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float f[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = bf16_lo_to_f32(w[i]);
+    f[2 * i + 1] = bf16_hi_to_f32(w[i]);
+  }
+  float q[8];
+  bool exact = d < 2.35098870e-38f;  // 2^-125: 1/d would not be a finite normal
+  if (!exact) {
+    const float y = __frcp_rn(d);
+    bool near = false;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      q[i] = __fmul_rn(f[i], y);
+      near |= near_e4m3_decision(q[i]);
+    }
+    exact = __any_sync(0xFFFFFFFFu, near);
+  }
+  if (exact) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], d);
+  }
+  return make_uint2(cvt_e4m3x2(q[1], q[0]) | (cvt_e4m3x2(q[3], q[2]) << 16),
+                    cvt_e4m3x2(q[5], q[4]) | (cvt_e4m3x2(q[7], q[6]) << 16));
 }
 
 // Loads 8 BF16 values at p (16-byte aligned); elements at or past `valid`
@@ -102,7 +135,8 @@ __global__ void __launch_bounds__(256) quantize_weight_kernel(
   for (int i = 0; i < 8; ++i) {
     const int c = tid + 256 * i;
     const int r = c >> 4, kk = (c & 15) * 8;
-    if (r < rows && kk < cols) store8_codes(q + (n0 + r) * ldq + k0 + kk, encode8(v[i], d), cols - kk);
+    const uint2 codes = encode8(v[i], d);  // every lane encodes (warp vote inside)
+    if (r < rows && kk < cols) store8_codes(q + (n0 + r) * ldq + k0 + kk, codes, cols - kk);
   }
 }
 
@@ -181,8 +215,8 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
   for (int off = 8; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
   const float amax = __uint_as_float(mx << 16);
   const float s = __fdiv_rn(amax, 448.0f);
-  const float d = (amax == 0.0f) ? 1.0f : s;
-  if (valid) store8_codes(qx + m * ldqx + k, encode8(v, d), nvalid);
+  const uint2 codes = encode8(v, (amax == 0.0f) ? 1.0f : s);  // every lane (warp vote)
+  if (valid) store8_codes(qx + m * ldqx + k, codes, nvalid);
   if (live && j == 0) sx[static_cast<int64_t>(kb) * ldsx + m] = s;
 }
 
