@@ -7,18 +7,28 @@
 // exactly representable in BF16, so the tensor cores see the exact weights.
 //
 // The product is computed transposed ("swap AB"): the 128 weight rows of a
-// CTA are the MMA's M dimension and the tokens its N dimension, so small
+// tile are the MMA's M dimension and the tokens its N dimension, so small
 // token counts still fill the 128-row MMA. A weight slab is expanded
 // FP8 -> BF16 once, straight into TMEM (the MMA's A operand), and used for
 // NSUB token sub-tiles of BT tokens each; the expansion costs no
 // shared-memory write traffic.
 //
+// Persistent kernel: one CTA per SM walks tiles (NSUB x BT tokens by 128
+// weight rows; token tiles of one weight tile are neighbours in the order,
+// so they share it through L2), and every ring runs on across tiles. The MMA
+// thread waits once for everything a slab needs, issues its MMAs back to
+// back and commits once per sub-tile group to a ring of "group done"
+// barriers that every consumer reads (the producer recycling activation
+// slots, the expansion warps recycling A buffers, the promotion warps
+// reading partials): commits and waits stall the tensor pipe, and one
+// commit per group lets promotion of a group start while the next one runs.
+//
 // Warp roles (16 warps; registers rebalanced per warpgroup with setmaxnreg):
 //   warp 0       TMA producer: weight-code slabs [128 x 128 B] into a q ring,
 //                activation sub-tiles [BT x 128 BF16] into an x ring;
-//   warp 1       TMEM allocator and MMA issuer: per slab and sub-tile,
-//                8 x (M=128, N=BT, K=16), A from TMEM, B from shared memory,
-//                into a 3-deep ring of TMEM partials;
+//   warp 1       TMEM allocator and MMA issuer: per slab NSUB x 8 x
+//                (M=128, N=BT, K=16), A from TMEM, B from shared memory, into
+//                a ring of TMEM partials;
 //   warps 4-7    expansion: one weight row per thread (TMEM lane), 128 codes
 //                -> 64 bf16x2 words -> tcgen05.st into one of two A buffers;
 //   warps 8-15   promotion/epilogue: warp (8 + 4t + q) owns TMEM lanes of
@@ -41,12 +51,13 @@ struct W8A16Cfg {
   static constexpr int QS = BT >= 128 ? 3 : (BT >= 64 ? 4 : 7);
   static constexpr int XS = BT >= 128 ? (NSUB == 2 ? 5 : 4) : (BT >= 64 ? 6 : 7);
   static constexpr int THREADS = 512;
-  static constexpr int PB = 3;                  // TMEM partial ring depth
+  static constexpr int PB = 3;                  // TMEM partial ring depth (items)
+  static constexpr int RD = 8;                  // "group done" barrier ring depth (items)
   static constexpr int TMEM_A = 0;              // 2 buffers x 64 columns
   static constexpr int TMEM_P = 128;            // PB buffers x BT columns
   static constexpr int TMEM_USED = TMEM_P + PB * BT;
   static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
-  static constexpr int NBAR = 2 * QS + 2 * XS + 4 + 2 * PB;
+  static constexpr int NBAR = 2 * QS + XS + 2 + RD + PB;
   static constexpr size_t SMEM_TILES =
       static_cast<size_t>(QS) * Q_BYTES + static_cast<size_t>(XS) * X_BYTES;
   static constexpr size_t SMEM = 1024 + SMEM_TILES + 8 * NBAR + 16;
@@ -55,6 +66,14 @@ struct W8A16Cfg {
   static_assert(NSUB == 1 || NSUB == 2, "sub-tiles");
   static_assert(TMEM_USED <= 512, "TMEM");
   static_assert(SMEM <= 227 * 1024, "shared memory");
+  // Item i = NSUB * slab + sub-tile. Every consumer of item i's "done"
+  // barrier waits on it before item i + RD can be committed: the producer
+  // recycles an x slot XS items later, the expansion waits for the last item
+  // of slab j - 2 before filling slab j's A buffer, and the MMA issues items
+  // in order and waits before item k for the promotion of item k - PB, so
+  // some item up to i + RD waits for a promotion (same sub-tile as i) that
+  // follows the wait on item i.
+  static_assert(RD >= XS && RD >= 2 * NSUB && RD - PB >= NSUB - 1, "done ring depth");
 };
 
 // Expand 16 E4M3 codes (one 16-byte chunk) into 8 bf16x2 words.
@@ -69,11 +88,16 @@ __device__ __forceinline__ void expand16(const uint4& c, uint32_t* o) {
   o[7] = e4m3x2_to_bf16x2(c.w >> 16);
 }
 
+__device__ __forceinline__ uint32_t ring_parity(int item, int depth) {
+  return static_cast<uint32_t>((item / depth) & 1);
+}
+
 template <int BT, int NSUB>
 __global__ void __launch_bounds__(512, 1)
     w8a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_x,
                       const float* __restrict__ sw, __nv_bfloat16* __restrict__ y, int64_t ldy,
-                      int M, int N, int KB, unsigned* __restrict__ err) {
+                      int M, int N, int KB, int mtiles, int ntiles_total,
+                      unsigned* __restrict__ err) {
   using C = W8A16Cfg<BT, NSUB>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
@@ -84,35 +108,26 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* qfull = bars;              // codes landed          (1 arrival + tx)
   uint64_t* qempty = qfull + C::QS;    // codes read            (4 expansion warps)
   uint64_t* xfull = qempty + C::QS;    // x sub-tile landed     (1 arrival + tx)
-  uint64_t* xempty = xfull + C::XS;    // x sub-tile consumed   (1 commit)
-  uint64_t* afull = xempty + C::XS;    // A buffer written      (4 expansion warps)
-  uint64_t* aempty = afull + 2;        // A buffer consumed     (1 commit)
-  uint64_t* pfull = aempty + 2;        // partial ready         (1 commit)
-  uint64_t* pempty = pfull + C::PB;    // partial consumed      (4 epilogue warps)
+  uint64_t* afull = xfull + C::XS;     // A buffer written      (4 expansion warps)
+  uint64_t* done = afull + 2;          // group's MMAs complete (1 commit)
+  uint64_t* pempty = done + C::RD;     // partial consumed      (4 epilogue warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + C::PB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // The token tiles of one weight tile are adjacent in the grid, so they run
-  // together and read the weight tile from DRAM once.
-  const int m0 = blockIdx.x * (BT * NSUB), n0 = blockIdx.y * 128;
+  // Slabs this CTA will run: KB per tile, tiles blockIdx.x, +gridDim.x, ...
+  const int my_tiles =
+      static_cast<int>(blockIdx.x) < ntiles_total ? (ntiles_total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int total_slabs = my_tiles * KB;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::QS; ++s) {
       mbar_init(&qfull[s], 1);
       mbar_init(&qempty[s], 4);
     }
-    for (int s = 0; s < C::XS; ++s) {
-      mbar_init(&xfull[s], 1);
-      mbar_init(&xempty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&afull[b], 4);
-      mbar_init(&aempty[b], 1);
-    }
-    for (int b = 0; b < C::PB; ++b) {
-      mbar_init(&pfull[b], 1);
-      mbar_init(&pempty[b], 4);
-    }
+    for (int s = 0; s < C::XS; ++s) mbar_init(&xfull[s], 1);
+    for (int b = 0; b < 2; ++b) mbar_init(&afull[b], 4);
+    for (int b = 0; b < C::RD; ++b) mbar_init(&done[b], 1);
+    for (int b = 0; b < C::PB; ++b) mbar_init(&pempty[b], 4);
     mbar_init_fence();
   }
   if (warp == 1) {
@@ -129,180 +144,180 @@ __global__ void __launch_bounds__(512, 1)
   const int wg = warp >> 2;
   if (wg == 0) {
     setmaxnreg_dec<56>();
-  if (warp == 0) {
-    if (lane == 0) {
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ producer
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_x);
-      Ring qr, xr;
-      int q_issued = 0, x_issued = 0;
+      int j = 0;  // slab counter (across tiles)
       bool ok = true;
-      for (int kb = 0; kb < KB && ok; ++kb) {
-        if (!mbar_wait(&qempty[qr.slot], qr.phase ^ 1u, err, kErrWaitLoad)) break;
-        mbar_arrive_expect_tx(&qfull[qr.slot], C::Q_BYTES);
-        tma_load_2d(sQ + qr.slot * C::Q_BYTES, &tm_q, &qfull[qr.slot], kb * 128, n0);
-        ++q_issued;
-        qr.next(C::QS);
-        for (int t = 0; t < NSUB; ++t) {
-          if (!mbar_wait(&xempty[xr.slot], xr.phase ^ 1u, err, kErrWaitLoad)) {
+      for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
+        const int m0 = (tile % mtiles) * (BT * NSUB), n0 = (tile / mtiles) * 128;
+        for (int kb = 0; kb < KB && ok; ++kb) {
+          const int qs = j % C::QS;
+          if (!mbar_wait_sleepy(&qempty[qs], ring_parity(j, C::QS) ^ 1u, err, kErrWaitLoad)) {
             ok = false;
             break;
           }
-          uint8_t* xs = sX + xr.slot * C::X_BYTES;
-          mbar_arrive_expect_tx(&xfull[xr.slot], C::X_BYTES);
-          tma_load_2d(xs, &tm_x, &xfull[xr.slot], kb * 128, m0 + t * BT);
-          tma_load_2d(xs + C::X_ATOM, &tm_x, &xfull[xr.slot], kb * 128 + 64, m0 + t * BT);
-          ++x_issued;
-          xr.next(C::XS);
+          mbar_arrive_expect_tx(&qfull[qs], C::Q_BYTES);
+          tma_load_2d(sQ + qs * C::Q_BYTES, &tm_q, &qfull[qs], kb * 128, n0);
+          for (int t = 0; t < NSUB; ++t) {
+            const int i = j * NSUB + t, xs = i % C::XS;
+            if (i >= C::XS) {  // the group that last used this slot has finished
+              const int io = i - C::XS;
+              if (!mbar_wait_sleepy(&done[io % C::RD], ring_parity(io, C::RD), err, kErrWaitLoad)) {
+                ok = false;
+                break;
+              }
+            }
+            uint8_t* xsm = sX + xs * C::X_BYTES;
+            mbar_arrive_expect_tx(&xfull[xs], C::X_BYTES);
+            tma_load_2d(xsm, &tm_x, &xfull[xs], kb * 128, m0 + t * BT);
+            tma_load_2d(xsm + C::X_ATOM, &tm_x, &xfull[xs], kb * 128 + 64, m0 + t * BT);
+          }
+          if (ok) ++j;
         }
       }
-      // Drain: the last load into every used slot has landed before exit.
+      // Drain: every load issued has landed before the CTA may exit. (On a
+      // time-out the slab in progress may have part of its loads issued; the
+      // drain waits, bounded, on the last phase of every slot touched.)
+      const int q_issued = ok ? j : j + 1, x_issued = ok ? j * NSUB : (j + 1) * NSUB;
       for (int s = 0; s < C::QS && s < q_issued; ++s)
         mbar_wait(&qfull[s], last_parity((q_issued - s + C::QS - 1) / C::QS), err, kErrWaitLoad);
       for (int s = 0; s < C::XS && s < x_issued; ++s)
         mbar_wait(&xfull[s], last_parity((x_issued - s + C::XS - 1) / C::XS), err, kErrWaitLoad);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ----------------------------------------------------------------- MMA
       // Descriptors are formed once; stepping through shared memory adds
       // (bytes >> 4) to their start-address field.
       const uint64_t xdesc0 = sw128_kmajor_desc(smem_addr(sX));
-      Ring xr, ar, pr;
-      int issued = 0, last_p = 0;
-      uint32_t last_phase = 0;
+      int i = 0;  // items issued
       bool ok = true;
-      for (int kb = 0; kb < KB && ok; ++kb) {
-        if (!mbar_wait(&afull[ar.slot], ar.phase, err, kErrWaitMma)) break;
-        const uint32_t a = tmem + static_cast<uint32_t>(C::TMEM_A + ar.slot * 64);
+      for (int j = 0; j < total_slabs && ok; ++j) {
+        if (!mbar_wait(&afull[j & 1], ring_parity(j, 2), err, kErrWaitMma)) break;
+        const uint32_t a = tmem + static_cast<uint32_t>(C::TMEM_A + (j & 1) * 64);
+#pragma unroll
         for (int t = 0; t < NSUB; ++t) {
-          if (!mbar_wait(&xfull[xr.slot], xr.phase, err, kErrWaitMma) ||
-              !mbar_wait(&pempty[pr.slot], pr.phase ^ 1u, err, kErrWaitMma)) {
-            ok = false;
-            break;
-          }
+          ok = mbar_wait(&xfull[i % C::XS], ring_parity(i, C::XS), err, kErrWaitMma) &&
+               (i < C::PB ||
+                mbar_wait(&pempty[i % C::PB], ring_parity(i - C::PB, C::PB), err, kErrWaitMma));
+          if (!ok) break;
           tc_fence_after_sync();
-          const uint64_t xd = xdesc0 + static_cast<uint64_t>((xr.slot * C::X_BYTES) >> 4);
-          const uint32_t d = tmem + static_cast<uint32_t>(C::TMEM_P + pr.slot * BT);
+          const uint64_t xd = xdesc0 + static_cast<uint64_t>(((i % C::XS) * C::X_BYTES) >> 4);
+          const uint32_t d = tmem + static_cast<uint32_t>(C::TMEM_P + (i % C::PB) * BT);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mma_f16_ts(d, a + 8u * k,
                        xd + static_cast<uint64_t>(((k >> 2) * C::X_ATOM + (k & 3) * 32) >> 4),
                        C::IDESC, k > 0 ? 1u : 0u);
-          tc_commit(&xempty[xr.slot]);
-          tc_commit(&pfull[pr.slot]);
-          last_p = pr.slot;
-          last_phase = pr.phase;
-          ++issued;
-          xr.next(C::XS);
-          pr.next(C::PB);
+          tc_commit(&done[i % C::RD]);
+          ++i;
         }
-        if (!ok) break;
-        tc_commit(&aempty[ar.slot]);
-        ar.next(2);
       }
       // Drain: all issued MMAs have completed before TMEM is released.
-      if (issued > 0) mbar_wait(&pfull[last_p], last_phase, err, kErrWaitMma);
+      if (i > 0) mbar_wait(&done[(i - 1) % C::RD], ring_parity(i - 1, C::RD), err, kErrWaitMma);
     }
-  }
   } else if (wg == 1) {
     // ---------------------------------------------------------- expansion
     setmaxnreg_dec<80>();
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // weight row within the tile == TMEM lane
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    Ring qr, ar;
-    for (int kb = 0; kb < KB; ++kb) {
-      if (!mbar_wait_warp(&qfull[qr.slot], qr.phase, err, kErrWaitExpand)) break;
+    for (int j = 0; j < total_slabs; ++j) {
+      const int qs = j % C::QS;
+      if (!mbar_wait_warp(&qfull[qs], ring_parity(j, C::QS), err, kErrWaitExpand)) break;
       // Row r of the 128-byte-swizzled slab: 16-byte chunk c sits at chunk
       // position c ^ (r & 7).
-      const uint8_t* qrow = sQ + qr.slot * C::Q_BYTES + r * 128;
+      const uint8_t* qrow = sQ + qs * C::Q_BYTES + r * 128;
       uint4 c[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        c[j] = *reinterpret_cast<const uint4*>(qrow + ((j ^ (r & 7)) << 4));
+      for (int u = 0; u < 4; ++u)
+        c[u] = *reinterpret_cast<const uint4*>(qrow + ((u ^ (r & 7)) << 4));
       uint32_t o[32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) expand16(c[j], o + 8 * j);
+      for (int u = 0; u < 4; ++u) expand16(c[u], o + 8 * u);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        c[j] = *reinterpret_cast<const uint4*>(qrow + (((4 + j) ^ (r & 7)) << 4));
+      for (int u = 0; u < 4; ++u)
+        c[u] = *reinterpret_cast<const uint4*>(qrow + (((4 + u) ^ (r & 7)) << 4));
       __syncwarp();
-      if (lane == 0) mbar_arrive(&qempty[qr.slot]);
-      qr.next(C::QS);
-      if (!mbar_wait_warp(&aempty[ar.slot], ar.phase ^ 1u, err, kErrWaitExpand)) break;
+      if (lane == 0) mbar_arrive(&qempty[qs]);
+      // A buffer (j & 1) was last read by slab j - 2 (its last group).
+      const int ia = NSUB * (j - 2) + NSUB - 1;
+      if (j >= 2 && !mbar_wait_warp(&done[ia % C::RD], ring_parity(ia, C::RD), err, kErrWaitExpand))
+        break;
       tc_fence_after_sync();
-      const uint32_t ta = t_lane + static_cast<uint32_t>(C::TMEM_A + ar.slot * 64);
+      const uint32_t ta = t_lane + static_cast<uint32_t>(C::TMEM_A + (j & 1) * 64);
       tmem_st32x32(ta, o);
       // tcgen05.st takes its source registers when it issues, so they can be
       // refilled with the second half.
 #pragma unroll
-      for (int j = 0; j < 4; ++j) expand16(c[j], o + 8 * j);
+      for (int u = 0; u < 4; ++u) expand16(c[u], o + 8 * u);
       tmem_st32x32(ta + 32u, o);
       tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[ar.slot]);
-      ar.next(2);
+      if (lane == 0) mbar_arrive(&afull[j & 1]);
     }
   } else {
     setmaxnreg_inc<184>();
     if (((warp - 8) >> 2) < NSUB) {
-    // -------------------------------------------------- promotion/epilogue
-    const int t = (warp - 8) >> 2;  // token sub-tile
-    const int quad = warp & 3;
-    const int n = n0 + quad * 32 + lane;
-    const float* sw_row = sw + static_cast<int64_t>(blockIdx.y) * KB;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::TMEM_P;
-    uint64_t acc[BT / 2];
+      // ------------------------------------------------ promotion/epilogue
+      const int t = (warp - 8) >> 2;  // token sub-tile
+      const int quad = warp & 3;
+      const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::TMEM_P;
+      int j = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
+        const int m0 = (tile % mtiles) * (BT * NSUB), n0 = (tile / mtiles) * 128;
+        const int n = n0 + quad * 32 + lane;
+        const float* sw_row = sw + static_cast<int64_t>(n0 >> 7) * KB;
+        uint64_t acc[BT / 2];
 #pragma unroll
-    for (int i = 0; i < BT / 2; ++i) acc[i] = 0ull;
-    // This sub-tile's partials are items t, t + NSUB, t + 2 NSUB, ... of the ring.
-    Ring pr;
-    for (int i = 0; i < t; ++i) pr.next(C::PB);
-    float s_next = __ldg(sw_row);
-    bool ok = true;
-    for (int kb = 0; kb < KB; ++kb) {
-      const float s = s_next;
-      if (kb + 1 < KB) s_next = __ldg(sw_row + kb + 1);
-      if (!mbar_wait_warp(&pfull[pr.slot], pr.phase, err, kErrWaitEpilogue)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after_sync();
-      const uint64_t s2 = pack_f32x2(s, s);
-      const uint32_t tp = t_lane + static_cast<uint32_t>(pr.slot * BT);
-      if constexpr (BT == 16) {
-        uint32_t p[16];
-        tmem_ld32x16(tp, p);
+        for (int e = 0; e < BT / 2; ++e) acc[e] = 0ull;
+        float s_next = __ldg(sw_row);
+        for (int kb = 0; kb < KB; ++kb, ++j) {
+          const float s = s_next;
+          if (kb + 1 < KB) s_next = __ldg(sw_row + kb + 1);
+          const int i = j * NSUB + t;
+          if (!mbar_wait_warp(&done[i % C::RD], ring_parity(i, C::RD), err, kErrWaitEpilogue)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint64_t s2 = pack_f32x2(s, s);
+          const uint32_t tp = t_lane + static_cast<uint32_t>((i % C::PB) * BT);
+          if constexpr (BT == 16) {
+            uint32_t p[16];
+            tmem_ld32x16(tp, p);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) ffma2(acc[i], pack_u32x2(p[2 * i], p[2 * i + 1]), s2);
-      } else {
+            for (int e = 0; e < 8; ++e) ffma2(acc[e], pack_u32x2(p[2 * e], p[2 * e + 1]), s2);
+          } else {
 #pragma unroll
-        for (int j = 0; j < BT / 32; ++j) {
-          uint32_t p[32];
-          tmem_ld32x32(tp + 32u * j, p);
+            for (int h = 0; h < BT / 32; ++h) {
+              uint32_t p[32];
+              tmem_ld32x32(tp + 32u * h, p);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            ffma2(acc[16 * j + i], pack_u32x2(p[2 * i], p[2 * i + 1]), s2);
+              for (int e = 0; e < 16; ++e)
+                ffma2(acc[16 * h + e], pack_u32x2(p[2 * e], p[2 * e + 1]), s2);
+            }
+          }
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pempty[i % C::PB]);
+        }
+        const int mt = m0 + t * BT;
+        if (ok && n < N && mt < M) {
+          uint16_t* ycol = reinterpret_cast<uint16_t*>(y) + n;
+          const int mcount = min(BT, M - mt);
+#pragma unroll
+          for (int e = 0; e < BT / 2; ++e) {
+            const uint32_t b2 = cvt_bf16x2_pair(acc[e]);
+            if (2 * e < mcount)
+              ycol[static_cast<int64_t>(mt + 2 * e) * ldy] = static_cast<uint16_t>(b2 & 0xFFFFu);
+            if (2 * e + 1 < mcount)
+              ycol[static_cast<int64_t>(mt + 2 * e + 1) * ldy] = static_cast<uint16_t>(b2 >> 16);
+          }
         }
       }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&pempty[pr.slot]);
-      for (int i = 0; i < NSUB; ++i) pr.next(C::PB);
-    }
-    const int mt = m0 + t * BT;
-    if (ok && n < N && mt < M) {
-      uint16_t* ycol = reinterpret_cast<uint16_t*>(y) + n;
-      const int mcount = min(BT, M - mt);
-#pragma unroll
-      for (int i = 0; i < BT / 2; ++i) {
-        const uint32_t b2 = cvt_bf16x2_pair(acc[i]);
-        if (2 * i < mcount)
-          ycol[static_cast<int64_t>(mt + 2 * i) * ldy] = static_cast<uint16_t>(b2 & 0xFFFFu);
-        if (2 * i + 1 < mcount)
-          ycol[static_cast<int64_t>(mt + 2 * i + 1) * ldy] = static_cast<uint16_t>(b2 >> 16);
-      }
-    }
     }
   }
 
@@ -328,10 +343,21 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
   auto kern = w8a16_gemm_kernel<BT, NSUB>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(cdiv(M, BT * NSUB)), static_cast<unsigned>(cdiv(N, 128)));
-  kern<<<grid, C::THREADS, C::SMEM, L.stream>>>(tq, tx, sw, reinterpret_cast<__nv_bfloat16*>(y),
-                                                ldy, static_cast<int>(M), static_cast<int>(N),
-                                                static_cast<int>(cdiv(K, 128)), L.err);
+  {
+    // The setmaxnreg split (64512 registers) needs 128 per thread at launch.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kern));
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * C::THREADS < 128 * (56 + 80 + 184 + 184)) return cudaErrorInvalidConfiguration;
+  }
+  const int64_t mtiles = cdiv(M, BT * NSUB), tiles = mtiles * cdiv(N, 128);
+  // Slab and item counters are 32-bit per CTA.
+  if (tiles * cdiv(K, 128) * NSUB > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  const int grid = static_cast<int>(tiles < L.num_sms ? tiles : L.num_sms);
+  kern<<<grid, C::THREADS, C::SMEM, L.stream>>>(
+      tq, tx, sw, reinterpret_cast<__nv_bfloat16*>(y), ldy, static_cast<int>(M),
+      static_cast<int>(N), static_cast<int>(cdiv(K, 128)), static_cast<int>(mtiles),
+      static_cast<int>(tiles), L.err);
   return cudaGetLastError();
 }
 
@@ -342,7 +368,6 @@ size_t w8a16_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
 cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                               int64_t ldq, const float* sw, uint16_t* y, int64_t ldy, int64_t M,
                               int64_t N, int64_t K, void*, size_t) {
-  if (cdiv(N, 128) > 65535) return cudaErrorInvalidValue;
   if (M <= 16) return launch_bt<16, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
   if (M <= 32) return launch_bt<32, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
   if (M <= 64) return launch_bt<64, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);

@@ -78,6 +78,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   }
 }
 
+// Bounded wait for a thread that is normally far ahead of the barrier it
+// waits on (a TMA producer): it sleeps between polls instead of spinning,
+// leaving issue slots to the other warps of its SM sub-partition.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t* bar, uint32_t parity, unsigned* err,
+                                                 unsigned flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+      __nanosleep(64);
+      if (mbar_try_wait(bar, parity)) return true;
+    }
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicOr(err, flag);
+      return false;
+    }
+  }
+}
+
 // Warp-uniform bounded wait: lane 0 polls, every lane gets the same answer
 // and the warp is converged afterwards (needed before .sync.aligned ops).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, unsigned* err,
@@ -141,6 +161,28 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+
+// 2-D tile store shared -> global (out-of-bounds parts of the box are not
+// written); completion tracked with bulk async-groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t c0,
+                                             int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_addr(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N committed store groups still read their shared source.
+template <int N>
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until all committed store groups have completed.
+__device__ __forceinline__ void tma_store_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Orders this thread's generic-proxy shared-memory writes before later

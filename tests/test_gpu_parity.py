@@ -166,7 +166,9 @@ def test_quantize_act_bit_exact(wl):
 
 # ---------------------------------------------------------------- linears
 LINEAR_FULL = [W.TINY, W.RAGGED, W.Workload("k130_n300", 50, 130, 300),
-               W.Workload("m200_k384_n640", 200, 384, 640, row_gain_sigma=0.5)]
+               W.Workload("m200_k384_n640", 200, 384, 640, row_gain_sigma=0.5),
+               W.Workload("m130_k256_n13", 130, 256, 13),
+               W.Workload("m40_k128_n5", 40, 128, 5)]
 LINEAR_SAMPLED = [W.QKV, W.O_PROJ, W.GATE_UP, W.DOWN, W.LINEAR_512, W.LARGE_4096, W.LARGE_16384]
 SMALL_M = [w.with_m(m) for w in W.DECODER_SHAPES for m in W.SMALL_M]
 
