@@ -199,10 +199,12 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
       uint64_t acc[64];  // column pairs
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = 0ull;
-      float c_next = has_cols ? __ldg(sx_col) * __ldg(sw_row) : 0.0f;
+      // The two scale factors of a slab are loaded one slab ahead and only
+      // multiplied when used, so the product does not wait on the loads.
+      float fx = has_cols ? __ldg(sx_col) : 0.0f, fw = has_cols ? __ldg(sw_row) : 0.0f;
       for (int kb = 0; kb < KB; ++kb, ++j) {
-        const float c = c_next;
-        if (has_cols && kb + 1 < KB) c_next = __ldg(sx_col + (kb + 1) * ldsx) * __ldg(sw_row + kb + 1);
+        const float c = fx * fw;
+        if (has_cols && kb + 1 < KB) { fx = __ldg(sx_col + (kb + 1) * ldsx); fw = __ldg(sw_row + kb + 1); }
         if (!mbar_wait_warp(&done[j & (C::RD - 1)], static_cast<uint32_t>((j / C::RD) & 1), err,
                             kErrWaitEpilogue)) {
           ok = false;

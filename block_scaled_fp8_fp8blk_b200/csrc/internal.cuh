@@ -35,11 +35,13 @@ cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, c
                               int64_t ldq, const float* scale_inv, uint16_t* y, int64_t ldy,
                               int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes);
 
-// 2-D tiled tensor map with 128-byte swizzling over a row-major matrix
-// [outer][inner] whose rows are row_bytes apart; out-of-bounds reads are
-// zero-filled. Returns false when the driver rejects the description.
+// 2-D tiled tensor map (128-byte swizzling unless stated) over a row-major
+// matrix [outer][inner] whose rows are row_bytes apart; out-of-bounds reads
+// are zero-filled and out-of-bounds parts of a store are dropped. Returns
+// false when the driver rejects the description.
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
-                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 
 // Sets the kernel's dynamic shared-memory limit once per device.
 cudaError_t ensure_smem_limit(const void* kernel, size_t bytes);

@@ -25,49 +25,72 @@ __device__ __forceinline__ uint32_t absmax_u4(uint32_t acc, const uint4& v) {
 // The codes are E4M3(RN_f32(v / d)): the float quotient (IEEE division,
 // round to nearest even) rounded again to E4M3 with saturation.
 //
-// Division is the converter's costliest step, so when d >= 2^-125 a cheaper
-// route gives the same codes: with y = RN(1 / d), q = RN(v * y) lies within a
-// few float ulps of RN(v / d). E4M3 rounding can only tell them apart near one
-// of its decision points -- floats whose low 20 mantissa bits are 0x80000
-// (midpoints of the 3-bit mantissa grid) -- or in E4M3's subnormal range;
-// when any element of a warp's chunk is there (|low20 - 0x80000| <= 16 ulps,
-// or 0 < |q| < 2^-5) the whole chunk takes the exact quotient instead (a
-// warp-uniform branch; rare for real data). Checked exhaustively against the
-// exact quotient over every BF16 value v and every BF16 block maximum
-// (d = amax / 448).
-__device__ __forceinline__ bool near_e4m3_decision(float q) {
-  const uint32_t b = __float_as_uint(q) & 0x7FFFFFFFu;
-  return b != 0u && (b < 0x3D000000u || ((b & 0xFFFFFu) - 0x7FFF0u) <= 0x20u);
+// Division is the converter's costliest step, so when d >= 2^-125 a bracket
+// gives the same codes from two products: with y = RN(1 / d),
+// ylo = RN(y (1 - 2^-21)) and yhi = RN(y (1 + 2^-21)), the products
+// RN(v ylo) and RN(v yhi) lie on either side of RN(v / d) (each of y, ylo,
+// RN(v ylo) adds at most 2^-24 relative error, 3 x 2^-24 < 2^-21 - 2^-24).
+// E4M3 rounding is monotone, so when both ends give the same code, so does
+// the quotient. When any element of a warp's chunk straddles a decision point
+// the whole chunk takes the exact quotient instead (a warp-uniform branch;
+// rare for real data). Checked exhaustively against the exact quotient over
+// every BF16 value v and every BF16 block maximum (d = amax / 448).
+struct E4M3Divisor {
+  float d;         // the divisor
+  uint64_t ylo2;   // RN(y (1 - 2^-21)) in both halves
+  uint64_t yhi2;   // RN(y (1 + 2^-21)) in both halves
+  bool exact;      // 1 / d is not a finite normal: always divide
+};
+
+__device__ __forceinline__ E4M3Divisor make_divisor(float d) {
+  E4M3Divisor r;
+  r.d = d;
+  r.exact = d < 2.35098870e-38f;  // 2^-125
+  const float y = __frcp_rn(r.exact ? 1.0f : d);
+  const float ylo = __fmul_rn(y, 0.99999952316284180f);  // 1 - 2^-21
+  const float yhi = __fmul_rn(y, 1.00000047683715820f);  // 1 + 2^-21
+  r.ylo2 = pack_f32x2(ylo, ylo);
+  r.yhi2 = pack_f32x2(yhi, yhi);
+  return r;
+}
+
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// E4M3 codes of the two floats packed in p (low half -> low byte).
+__device__ __forceinline__ uint32_t cvt_e4m3x2_packed(uint64_t p) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+  return cvt_e4m3x2(hi, lo);
 }
 
 // Eight BF16 values -> eight E4M3 codes of RN_f32(v / d) (code i in byte i).
 // All 32 lanes of the warp must call this together.
-__device__ __forceinline__ uint2 encode8(const uint4& v, float d) {
+__device__ __forceinline__ uint2 encode8(const uint4& v, const E4M3Divisor& dv) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float f[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = bf16_lo_to_f32(w[i]);
-    f[2 * i + 1] = bf16_hi_to_f32(w[i]);
-  }
-  float q[8];
-  bool exact = d < 2.35098870e-38f;  // 2^-125: 1/d would not be a finite normal
+  uint32_t code[4];
+  bool exact = dv.exact;
   if (!exact) {
-    const float y = __frcp_rn(d);
-    bool near = false;
+    uint32_t diff = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      q[i] = __fmul_rn(f[i], y);
-      near |= near_e4m3_decision(q[i]);
+    for (int i = 0; i < 4; ++i) {
+      const uint64_t f2 = pack_u32x2(w[i] << 16, w[i] & 0xFFFF0000u);
+      const uint32_t clo = cvt_e4m3x2_packed(fmul2(f2, dv.ylo2));
+      const uint32_t chi = cvt_e4m3x2_packed(fmul2(f2, dv.yhi2));
+      diff |= clo ^ chi;
+      code[i] = clo;
     }
-    exact = __any_sync(0xFFFFFFFFu, near);
+    exact = __any_sync(0xFFFFFFFFu, diff != 0u);
   }
   if (exact) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], d);
+    for (int i = 0; i < 4; ++i)
+      code[i] = cvt_e4m3x2(__fdiv_rn(bf16_hi_to_f32(w[i]), dv.d), __fdiv_rn(bf16_lo_to_f32(w[i]), dv.d));
   }
-  return make_uint2(cvt_e4m3x2(q[1], q[0]) | (cvt_e4m3x2(q[3], q[2]) << 16),
-                    cvt_e4m3x2(q[5], q[4]) | (cvt_e4m3x2(q[7], q[6]) << 16));
+  return make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
 }
 
 // Loads 8 BF16 values at p (16-byte aligned); elements at or past `valid`
@@ -92,51 +115,111 @@ __device__ __forceinline__ void store8_codes(uint8_t* p, uint2 c, int valid) {
 }
 
 // ------------------------------------------------------------- converter
-// One CTA per 128 x 128 block (FastVideo PR #1829, "Changes", converter
-// bullet): 256 threads x 8 chunks of 8 BF16 values stay in registers; the
-// block amax is reduced across the CTA; every element is then divided by
-// s = amax / 448 and encoded.
-__global__ void __launch_bounds__(256) quantize_weight_kernel(
-    const uint16_t* __restrict__ w, int64_t N, int64_t K, int64_t ldw, uint8_t* __restrict__ q,
-    int64_t ldq, float* __restrict__ scale_inv, int KB) {
-  const int64_t blk = blockIdx.x;
-  const int64_t nb = blk / KB, kb = blk - nb * KB;
-  const int64_t n0 = nb * 128, k0 = kb * 128;
-  const int rows = static_cast<int>((N - n0 < 128 ? N - n0 : 128));
-  const int cols = static_cast<int>((K - k0 < 128 ? K - k0 : 128));
+// Per 128 x 128 block (FastVideo PR #1829, "Changes", converter bullet): the
+// block amax over the BF16 values, s = amax / 448, and every element divided
+// by s and encoded. Persistent CTAs (two per SM) walk the blocks b =
+// blockIdx.x, + gridDim.x, ... in row-major block order. Thread 0 keeps a
+// 3-deep ring of TMA loads in flight (box 128 x 128 BF16, unswizzled; parts
+// past N or K read as 0, which never changes an amax). Each of the eight
+// warps takes 16 rows of a block: lane l reads elements 4l..4l+3 of each row
+// (8-byte shared loads, conflict-free), the warps' maxima meet in shared
+// memory, and each lane then encodes its 64 values and writes 4 codes per row
+// (128 contiguous bytes per warp and row). Once the amax barrier is passed
+// every warp has read the stage, so thread 0 refills it right away.
+constexpr int kCvtStages = 3;
+constexpr int kCvtStageBytes = 128 * 128 * 2;
+constexpr size_t kCvtSmem = 128 + static_cast<size_t>(kCvtStages) * kCvtStageBytes;
+
+__global__ void __launch_bounds__(256, 2) quantize_weight_kernel(
+    const __grid_constant__ CUtensorMap tm_w, int64_t N, int64_t K, uint8_t* __restrict__ q,
+    int64_t ldq, float* __restrict__ scale_inv, int KB, int nblocks, unsigned* __restrict__ err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
+  __shared__ uint64_t full[kCvtStages];
+  __shared__ uint32_t red[2][8];
+  __shared__ int abort_flag;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  uint4 v[8];
-  uint32_t m2 = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int c = tid + 256 * i;
-    const int r = c >> 4, kk = (c & 15) * 8;
-    v[i] = make_uint4(0, 0, 0, 0);
-    if (r < rows && kk < cols) v[i] = load8_bf16(w + (n0 + r) * ldw + k0 + kk, cols - kk);
-    m2 = absmax_u4(m2, v[i]);
+  if (tid == 0) {
+    for (int s = 0; s < kCvtStages; ++s) mbar_init(&full[s], 1);
+    mbar_init_fence();
+    abort_flag = 0;
   }
-  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
-  m = __reduce_max_sync(0xFFFFFFFFu, m);
-  __shared__ uint32_t red[8];
-  if (lane == 0) red[warp] = m;
   __syncthreads();
-  m = red[0];
+  // Thread 0: load this CTA's i-th block into stage i % kCvtStages.
+  auto issue = [&](int i) {
+    const int b = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    if (b >= nblocks) return;
+    const int nb = b / KB, kb = b - nb * KB;
+    uint64_t* bar = &full[i % kCvtStages];
+    mbar_arrive_expect_tx(bar, kCvtStageBytes);
+    tma_load_2d(smem + (i % kCvtStages) * kCvtStageBytes, &tm_w, bar, kb * 128, nb * 128);
+  };
+  if (tid == 0) {
+    tma_prefetch_map(&tm_w);
+    for (int i = 0; i < kCvtStages; ++i) issue(i);
+  }
+  int i = 0;
+  for (;; ++i) {
+    const int b = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    if (b >= nblocks) break;
+    const int st = i % kCvtStages;
+    const bool landed = mbar_wait_warp(&full[st], static_cast<uint32_t>((i / kCvtStages) & 1), err,
+                                       kErrWaitLoad);
+    const uint8_t* rows16 = smem + st * kCvtStageBytes + warp * 16 * 256 + lane * 8;
+    uint2 v[16];
+    uint32_t m2 = 0;
 #pragma unroll
-  for (int i = 1; i < 8; ++i) m = max(m, red[i]);
-
-  const float amax = __uint_as_float(m << 16);
-  const float s = __fdiv_rn(amax, 448.0f);
-  if (tid == 0) scale_inv[blk] = s;
-  // An all-zero block has s = 0: its +-0 elements keep their sign under a
-  // division by 1 instead.
-  const float d = (amax == 0.0f) ? 1.0f : s;
+    for (int r = 0; r < 16; ++r) {
+      v[r] = *reinterpret_cast<const uint2*>(rows16 + r * 256);
+      m2 = absmax2(absmax2(m2, v[r].x), v[r].y);
+    }
+    uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+    if (lane == 0) {
+      red[i & 1][warp] = m;
+      if (!landed) abort_flag = 1;
+    }
+    __syncthreads();
+    if (abort_flag) break;
+    if (tid == 0) issue(i + kCvtStages);  // every warp has read this stage
+    m = red[i & 1][0];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int c = tid + 256 * i;
-    const int r = c >> 4, kk = (c & 15) * 8;
-    const uint2 codes = encode8(v[i], d);  // every lane encodes (warp vote inside)
-    if (r < rows && kk < cols) store8_codes(q + (n0 + r) * ldq + k0 + kk, codes, cols - kk);
+    for (int w = 1; w < 8; ++w) m = max(m, red[i & 1][w]);
+    const float amax = __uint_as_float(m << 16);
+    const float s = __fdiv_rn(amax, 448.0f);
+    if (tid == 0) scale_inv[b] = s;
+    // An all-zero block has s = 0: its +-0 elements keep their sign under a
+    // division by 1 instead.
+    const E4M3Divisor dv = make_divisor((amax == 0.0f) ? 1.0f : s);
+    const int nb = b / KB, kb = b - nb * KB;
+    const int64_t n0 = static_cast<int64_t>(nb) * 128, k0 = static_cast<int64_t>(kb) * 128;
+    const int rows = static_cast<int>(N - n0 < 128 ? N - n0 : 128);
+    const int cols = static_cast<int>(K - k0 < 128 ? K - k0 : 128);
+    const int col = 4 * lane;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      // rows 2g and 2g + 1 of this warp's 16: every lane encodes (warp vote inside)
+      const uint2 c = encode8(make_uint4(v[2 * g].x, v[2 * g].y, v[2 * g + 1].x, v[2 * g + 1].y), dv);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = warp * 16 + 2 * g + h;
+        const uint32_t codes = h ? c.y : c.x;
+        if (r < rows && col < cols) {
+          uint8_t* dst = q + (n0 + r) * ldq + k0 + col;
+          if (col + 4 <= cols) {
+            __stcs(reinterpret_cast<unsigned int*>(dst), codes);
+          } else {
+            for (int t = 0; t < cols - col; ++t) dst[t] = static_cast<uint8_t>(codes >> (8 * t));
+          }
+        }
+      }
+    }
+  }
+  // After a time-out, the loads still in flight land before the CTA exits.
+  if (tid == 0 && abort_flag) {
+    for (int k = i; k < i + kCvtStages; ++k) {
+      const int b = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+      if (b < nblocks) mbar_wait(&full[k % kCvtStages], static_cast<uint32_t>((k / kCvtStages) & 1), err, kErrWaitLoad);
+    }
   }
 }
 
@@ -215,7 +298,7 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
   for (int off = 8; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
   const float amax = __uint_as_float(mx << 16);
   const float s = __fdiv_rn(amax, 448.0f);
-  const uint2 codes = encode8(v, (amax == 0.0f) ? 1.0f : s);  // every lane (warp vote)
+  const uint2 codes = encode8(v, make_divisor((amax == 0.0f) ? 1.0f : s));  // every lane (warp vote)
   if (valid) store8_codes(qx + m * ldqx + k, codes, nvalid);
   if (live && j == 0) sx[static_cast<int64_t>(kb) * ldsx + m] = s;
 }
@@ -248,8 +331,16 @@ cudaError_t launch_quantize_weight(const Launch& L, const uint16_t* w, int64_t N
                                    int64_t ldw, uint8_t* q, int64_t ldq, float* scale_inv) {
   const int64_t NB = cdiv(N, 128), KB = cdiv(K, 128);
   if (NB * KB > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  quantize_weight_kernel<<<static_cast<unsigned>(NB * KB), 256, 0, L.stream>>>(
-      w, N, K, ldw, q, ldq, scale_inv, static_cast<int>(KB));
+  CUtensorMap tw;
+  if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, N, 2 * ldw, 128, 128,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(quantize_weight_kernel), kCvtSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t nblocks = NB * KB, cap = 2 * static_cast<int64_t>(L.num_sms);
+  quantize_weight_kernel<<<static_cast<unsigned>(nblocks < cap ? nblocks : cap), 256, kCvtSmem,
+                           L.stream>>>(tw, N, K, q, ldq, scale_inv, static_cast<int>(KB),
+                                       static_cast<int>(nblocks), L.err);
   return cudaGetLastError();
 }
 
