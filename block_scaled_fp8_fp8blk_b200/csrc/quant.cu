@@ -31,10 +31,9 @@ __device__ __forceinline__ uint32_t absmax_u4(uint32_t acc, const uint4& v) {
 // RN(v ylo) and RN(v yhi) lie on either side of RN(v / d) (each of y, ylo,
 // RN(v ylo) adds at most 2^-24 relative error, 3 x 2^-24 < 2^-21 - 2^-24).
 // E4M3 rounding is monotone, so when both ends give the same code, so does
-// the quotient. When any element of a warp's chunk straddles a decision point
-// the whole chunk takes the exact quotient instead (a warp-uniform branch;
-// rare for real data). Checked exhaustively against the exact quotient over
-// every BF16 value v and every BF16 block maximum (d = amax / 448).
+// the quotient; elements whose bracket straddles a decision point take the
+// exact quotient instead. Checked exhaustively against the exact quotient
+// over every BF16 value v and every BF16 block maximum (d = amax / 448).
 struct E4M3Divisor {
   float d;         // the divisor
   uint64_t ylo2;   // RN(y (1 - 2^-21)) in both halves
@@ -68,27 +67,37 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2_packed(uint64_t p) {
 }
 
 // Eight BF16 values -> eight E4M3 codes of RN_f32(v / d) (code i in byte i).
-// All 32 lanes of the warp must call this together.
+// All 32 lanes of the warp must call this together. Element positions where
+// some lane's bracket straddles a decision point take the exact quotient
+// (for the other lanes it gives the same code); BF16 data hit such near-ties
+// often, since v / (amax / 448) is a ratio of two 8-bit mantissas times 7.
 __device__ __forceinline__ uint2 encode8(const uint4& v, const E4M3Divisor& dv) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t code[4];
-  bool exact = dv.exact;
-  if (!exact) {
-    uint32_t diff = 0;
+  uint32_t code[4], diff[4];
+  if (dv.exact) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      diff[i] = 0xFFFFu;
+      code[i] = 0u;
+    }
+  } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint64_t f2 = pack_u32x2(w[i] << 16, w[i] & 0xFFFF0000u);
       const uint32_t clo = cvt_e4m3x2_packed(fmul2(f2, dv.ylo2));
       const uint32_t chi = cvt_e4m3x2_packed(fmul2(f2, dv.yhi2));
-      diff |= clo ^ chi;
+      diff[i] = clo ^ chi;
       code[i] = clo;
     }
-    exact = __any_sync(0xFFFFFFFFu, diff != 0u);
   }
-  if (exact) {
+  if (__any_sync(0xFFFFFFFFu, (diff[0] | diff[1] | diff[2] | diff[3]) != 0u)) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      code[i] = cvt_e4m3x2(__fdiv_rn(bf16_hi_to_f32(w[i]), dv.d), __fdiv_rn(bf16_lo_to_f32(w[i]), dv.d));
+    for (int i = 0; i < 4; ++i) {
+      if (__any_sync(0xFFFFFFFFu, (diff[i] & 0xFFu) != 0u))
+        code[i] = (code[i] & 0xFF00u) | (cvt_e4m3x2(0.0f, __fdiv_rn(bf16_lo_to_f32(w[i]), dv.d)) & 0xFFu);
+      if (__any_sync(0xFFFFFFFFu, (diff[i] >> 8) != 0u))
+        code[i] = (code[i] & 0x00FFu) | (cvt_e4m3x2(__fdiv_rn(bf16_hi_to_f32(w[i]), dv.d), 0.0f) & 0xFF00u);
+    }
   }
   return make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
 }
