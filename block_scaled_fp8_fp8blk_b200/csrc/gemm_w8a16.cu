@@ -15,20 +15,20 @@
 //
 // Persistent kernel: one CTA per SM walks tiles (NSUB x BT tokens by 128
 // weight rows; token tiles of one weight tile are neighbours in the order,
-// so they share it through L2), and every ring runs on across tiles. The MMA
-// thread waits once for everything a slab needs, issues its MMAs back to
-// back and commits once per sub-tile group to a ring of "group done"
-// barriers that every consumer reads (the producer recycling activation
-// slots, the expansion warps recycling A buffers, the promotion warps
-// reading partials): commits and waits stall the tensor pipe, and one
-// commit per group lets promotion of a group start while the next one runs.
+// so they share it through L2), and every ring runs on across tiles. Each
+// sub-tile group ("item" i = NSUB * slab + t) is issued and committed by its
+// own MMA thread to a ring of "item done" barriers that every consumer reads
+// (the activation producer recycling slots, the expansion warps recycling A
+// buffers, the promotion warps reading partials): a commit stalls its
+// issuer's MMA stream for a few hundred cycles, and with one issuer per
+// sub-tile the other issuer's MMAs fill that gap.
 //
 // Warp roles (16 warps; registers rebalanced per warpgroup with setmaxnreg):
-//   warp 0       TMA producer: weight-code slabs [128 x 128 B] into a q ring,
-//                activation sub-tiles [BT x 128 BF16] into an x ring;
-//   warp 1       TMEM allocator and MMA issuer: per slab NSUB x 8 x
-//                (M=128, N=BT, K=16), A from TMEM, B from shared memory, into
-//                a ring of TMEM partials;
+//   warp 0       TMA producer of weight-code slabs [128 x 128 B] (q ring);
+//   warp 1       TMA producer of activation sub-tiles [BT x 128 BF16] (x ring);
+//   warps 2..    MMA issuers, one per sub-tile t: per slab 8 x (M=128, N=BT,
+//                K=16), A from TMEM, B from shared memory, into a ring of TMEM
+//                partials shared in item order (warp 2 also allocates TMEM);
 //   warps 4-7    expansion: one weight row per thread (TMEM lane), 128 codes
 //                -> 64 bf16x2 words -> tcgen05.st into one of two A buffers;
 //   warps 8-15   promotion/epilogue: warp (8 + 4t + q) owns TMEM lanes of
@@ -67,12 +67,17 @@ struct W8A16Cfg {
   static_assert(TMEM_USED <= 512, "TMEM");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   // Item i = NSUB * slab + sub-tile. Every consumer of item i's "done"
-  // barrier waits on it before item i + RD can be committed: the producer
-  // recycles an x slot XS items later, the expansion waits for the last item
-  // of slab j - 2 before filling slab j's A buffer, and the MMA issues items
-  // in order and waits before item k for the promotion of item k - PB, so
-  // some item up to i + RD waits for a promotion (same sub-tile as i) that
-  // follows the wait on item i.
+  // barrier waits on it before item i + RD can be committed. The activation
+  // producer recycles an x slot XS items later (RD >= XS keeps the loads of
+  // item i + RD behind its wait on item i). The expansion waits for the items
+  // of slab j - 2 before filling slab j's A buffer. The promotion warps of
+  // sub-tile t release a partial after waiting on its item; partials are used
+  // in item order across both issuers, so item k waits for the promotion of
+  // item k - PB, and with PB = 3 and two issuers each issuer waits on the
+  // other sub-tile's promotions: item i + RD needs the A buffer of slab
+  // (i + RD) / NSUB, whose expansion waited for both items of an earlier
+  // slab, one of which waited for the promotion of an item of sub-tile t at
+  // or after i (checked for RD = 8, PB = 3, NSUB <= 2).
   static_assert(RD >= XS && RD >= 2 * NSUB && RD - PB >= NSUB - 1, "done ring depth");
 };
 
@@ -130,7 +135,7 @@ __global__ void __launch_bounds__(512, 1)
     for (int b = 0; b < C::PB; ++b) mbar_init(&pempty[b], 4);
     mbar_init_fence();
   }
-  if (warp == 1) {
+  if (warp == 2) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -145,14 +150,13 @@ __global__ void __launch_bounds__(512, 1)
   if (wg == 0) {
     setmaxnreg_dec<56>();
     if (warp == 0 && lane == 0) {
-      // ------------------------------------------------------------ producer
+      // ------------------------------------------------ weight-code producer
       tma_prefetch_map(&tm_q);
-      tma_prefetch_map(&tm_x);
       int j = 0;  // slab counter (across tiles)
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
-        const int m0 = (tile % mtiles) * (BT * NSUB), n0 = (tile / mtiles) * 128;
-        for (int kb = 0; kb < KB && ok; ++kb) {
+        const int n0 = (tile / mtiles) * 128;
+        for (int kb = 0; kb < KB; ++kb, ++j) {
           const int qs = j % C::QS;
           if (!mbar_wait_sleepy(&qempty[qs], ring_parity(j, C::QS) ^ 1u, err, kErrWaitLoad)) {
             ok = false;
@@ -160,9 +164,22 @@ __global__ void __launch_bounds__(512, 1)
           }
           mbar_arrive_expect_tx(&qfull[qs], C::Q_BYTES);
           tma_load_2d(sQ + qs * C::Q_BYTES, &tm_q, &qfull[qs], kb * 128, n0);
-          for (int t = 0; t < NSUB; ++t) {
-            const int i = j * NSUB + t, xs = i % C::XS;
-            if (i >= C::XS) {  // the group that last used this slot has finished
+        }
+      }
+      // Drain: every load issued has landed before the CTA may exit.
+      for (int s = 0; s < C::QS && s < j; ++s)
+        mbar_wait(&qfull[s], last_parity((j - s + C::QS - 1) / C::QS), err, kErrWaitLoad);
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------- activation producer
+      tma_prefetch_map(&tm_x);
+      int i = 0;  // item counter (across tiles)
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
+        const int m0 = (tile % mtiles) * (BT * NSUB);
+        for (int kb = 0; kb < KB && ok; ++kb) {
+          for (int t = 0; t < NSUB; ++t, ++i) {
+            const int xs = i % C::XS;
+            if (i >= C::XS) {  // the item that last used this slot has finished
               const int io = i - C::XS;
               if (!mbar_wait_sleepy(&done[io % C::RD], ring_parity(io, C::RD), err, kErrWaitLoad)) {
                 ok = false;
@@ -174,47 +191,39 @@ __global__ void __launch_bounds__(512, 1)
             tma_load_2d(xsm, &tm_x, &xfull[xs], kb * 128, m0 + t * BT);
             tma_load_2d(xsm + C::X_ATOM, &tm_x, &xfull[xs], kb * 128 + 64, m0 + t * BT);
           }
-          if (ok) ++j;
         }
       }
-      // Drain: every load issued has landed before the CTA may exit. (On a
-      // time-out the slab in progress may have part of its loads issued; the
-      // drain waits, bounded, on the last phase of every slot touched.)
-      const int q_issued = ok ? j : j + 1, x_issued = ok ? j * NSUB : (j + 1) * NSUB;
-      for (int s = 0; s < C::QS && s < q_issued; ++s)
-        mbar_wait(&qfull[s], last_parity((q_issued - s + C::QS - 1) / C::QS), err, kErrWaitLoad);
-      for (int s = 0; s < C::XS && s < x_issued; ++s)
-        mbar_wait(&xfull[s], last_parity((x_issued - s + C::XS - 1) / C::XS), err, kErrWaitLoad);
-    } else if (warp == 1 && lane == 0) {
-      // ----------------------------------------------------------------- MMA
-      // Descriptors are formed once; stepping through shared memory adds
-      // (bytes >> 4) to their start-address field.
+      for (int s = 0; s < C::XS && s < i; ++s)
+        mbar_wait(&xfull[s], last_parity((i - s + C::XS - 1) / C::XS), err, kErrWaitLoad);
+    } else if (warp >= 2 && warp < 2 + NSUB && lane == 0) {
+      // ------------------------------------------------------- MMA issuers
+      // Issuer t runs the items of sub-tile t; with two issuers one's waits
+      // and commits hide behind the other's MMAs. Descriptors are formed
+      // once; stepping through shared memory adds (bytes >> 4) to their
+      // start-address field.
+      const int t = warp - 2;
       const uint64_t xdesc0 = sw128_kmajor_desc(smem_addr(sX));
-      int i = 0;  // items issued
-      bool ok = true;
-      for (int j = 0; j < total_slabs && ok; ++j) {
+      int last = -1;
+      for (int j = 0; j < total_slabs; ++j) {
+        const int i = j * NSUB + t;
         if (!mbar_wait(&afull[j & 1], ring_parity(j, 2), err, kErrWaitMma)) break;
+        if (!mbar_wait(&xfull[i % C::XS], ring_parity(i, C::XS), err, kErrWaitMma)) break;
+        if (i >= C::PB && !mbar_wait(&pempty[i % C::PB], ring_parity(i - C::PB, C::PB), err, kErrWaitMma))
+          break;
+        tc_fence_after_sync();
         const uint32_t a = tmem + static_cast<uint32_t>(C::TMEM_A + (j & 1) * 64);
+        const uint64_t xd = xdesc0 + static_cast<uint64_t>(((i % C::XS) * C::X_BYTES) >> 4);
+        const uint32_t d = tmem + static_cast<uint32_t>(C::TMEM_P + (i % C::PB) * BT);
 #pragma unroll
-        for (int t = 0; t < NSUB; ++t) {
-          ok = mbar_wait(&xfull[i % C::XS], ring_parity(i, C::XS), err, kErrWaitMma) &&
-               (i < C::PB ||
-                mbar_wait(&pempty[i % C::PB], ring_parity(i - C::PB, C::PB), err, kErrWaitMma));
-          if (!ok) break;
-          tc_fence_after_sync();
-          const uint64_t xd = xdesc0 + static_cast<uint64_t>(((i % C::XS) * C::X_BYTES) >> 4);
-          const uint32_t d = tmem + static_cast<uint32_t>(C::TMEM_P + (i % C::PB) * BT);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_f16_ts(d, a + 8u * k,
-                       xd + static_cast<uint64_t>(((k >> 2) * C::X_ATOM + (k & 3) * 32) >> 4),
-                       C::IDESC, k > 0 ? 1u : 0u);
-          tc_commit(&done[i % C::RD]);
-          ++i;
-        }
+        for (int k = 0; k < 8; ++k)
+          mma_f16_ts(d, a + 8u * k,
+                     xd + static_cast<uint64_t>(((k >> 2) * C::X_ATOM + (k & 3) * 32) >> 4),
+                     C::IDESC, k > 0 ? 1u : 0u);
+        tc_commit(&done[i % C::RD]);
+        last = i;
       }
-      // Drain: all issued MMAs have completed before TMEM is released.
-      if (i > 0) mbar_wait(&done[(i - 1) % C::RD], ring_parity(i - 1, C::RD), err, kErrWaitMma);
+      // Drain: this issuer's MMAs have completed before TMEM is released.
+      if (last >= 0) mbar_wait(&done[last % C::RD], ring_parity(last, C::RD), err, kErrWaitMma);
     }
   } else if (wg == 1) {
     // ---------------------------------------------------------- expansion
@@ -240,10 +249,16 @@ __global__ void __launch_bounds__(512, 1)
         c[u] = *reinterpret_cast<const uint4*>(qrow + (((4 + u) ^ (r & 7)) << 4));
       __syncwarp();
       if (lane == 0) mbar_arrive(&qempty[qs]);
-      // A buffer (j & 1) was last read by slab j - 2 (its last group).
-      const int ia = NSUB * (j - 2) + NSUB - 1;
-      if (j >= 2 && !mbar_wait_warp(&done[ia % C::RD], ring_parity(ia, C::RD), err, kErrWaitExpand))
-        break;
+      // A buffer (j & 1) was last read by the items of slab j - 2.
+      bool free_a = true;
+      if (j >= 2) {
+#pragma unroll
+        for (int t = 0; t < NSUB; ++t) {
+          const int ia = NSUB * (j - 2) + t;
+          free_a = free_a && mbar_wait_warp(&done[ia % C::RD], ring_parity(ia, C::RD), err, kErrWaitExpand);
+        }
+      }
+      if (!free_a) break;
       tc_fence_after_sync();
       const uint32_t ta = t_lane + static_cast<uint32_t>(C::TMEM_A + (j & 1) * 64);
       tmem_st32x32(ta, o);
@@ -323,7 +338,7 @@ __global__ void __launch_bounds__(512, 1)
 
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 2) {
     __syncwarp();
     tc_fence_after_sync();
     tmem_dealloc(tmem, C::TMEM_COLS);
