@@ -57,9 +57,10 @@ struct W8A16Cfg {
   static constexpr int TMEM_P = 128;            // PB buffers x BT columns
   static constexpr int TMEM_USED = TMEM_P + PB * BT;
   static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
-  static constexpr int NBAR = 2 * QS + XS + 2 + RD + PB;
-  static constexpr size_t SMEM_TILES =
-      static_cast<size_t>(QS) * Q_BYTES + static_cast<size_t>(XS) * X_BYTES;
+  static constexpr int NBAR = 2 * QS + XS + 2 + RD + PB * NSUB;
+  static constexpr int OUT_BYTES = 16 * 64;     // per epilogue warp: 16 tokens x 32 BF16
+  static constexpr size_t SMEM_TILES = static_cast<size_t>(QS) * Q_BYTES +
+                                       static_cast<size_t>(XS) * X_BYTES + 4 * NSUB * OUT_BYTES;
   static constexpr size_t SMEM = 1024 + SMEM_TILES + 8 * NBAR + 16;
   static constexpr uint32_t IDESC = make_idesc(1u, 1u, 128, BT);  // BF16 x BF16 -> F32
   static_assert(BT % 16 == 0 && BT >= 16 && BT <= 128, "MMA N for M=128");
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* smem = smem_raw + pad;
   uint8_t* sQ = smem;                       // QS x Q_BYTES
   uint8_t* sX = smem + C::QS * C::Q_BYTES;  // XS x X_BYTES
+  uint8_t* sOut = sX + C::XS * C::X_BYTES;  // 4 NSUB x OUT_BYTES output transposition
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_TILES);
   uint64_t* qfull = bars;              // codes landed          (1 arrival + tx)
   uint64_t* qempty = qfull + C::QS;    // codes read            (4 expansion warps)
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* afull = xfull + C::XS;     // A buffer written      (4 expansion warps)
   uint64_t* done = afull + 2;          // group's MMAs complete (1 commit)
   uint64_t* pempty = done + C::RD;     // partial consumed      (4 epilogue warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + C::PB);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + C::PB * NSUB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Slabs this CTA will run: KB per tile, tiles blockIdx.x, +gridDim.x, ...
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(512, 1)
     for (int s = 0; s < C::XS; ++s) mbar_init(&xfull[s], 1);
     for (int b = 0; b < 2; ++b) mbar_init(&afull[b], 4);
     for (int b = 0; b < C::RD; ++b) mbar_init(&done[b], 1);
-    for (int b = 0; b < C::PB; ++b) mbar_init(&pempty[b], 4);
+    for (int b = 0; b < C::PB * NSUB; ++b) mbar_init(&pempty[b], 4);
     mbar_init_fence();
   }
   if (warp == 2) {
@@ -208,8 +210,16 @@ __global__ void __launch_bounds__(512, 1)
         const int i = j * NSUB + t;
         if (!mbar_wait(&afull[j & 1], ring_parity(j, 2), err, kErrWaitMma)) break;
         if (!mbar_wait(&xfull[i % C::XS], ring_parity(i, C::XS), err, kErrWaitMma)) break;
-        if (i >= C::PB && !mbar_wait(&pempty[i % C::PB], ring_parity(i - C::PB, C::PB), err, kErrWaitMma))
-          break;
+        // Partial slot i % PB last held item k = i - PB, whose promotion
+        // arrives on that slot's barrier for k's sub-tile. Each issuer meets
+        // every phase of the barriers it waits on, in order (a parity wait
+        // cannot tell a phase from the one two before or after).
+        if (i >= C::PB) {
+          const int k = i - C::PB;
+          if (!mbar_wait(&pempty[(k % C::PB) * NSUB + k % NSUB], ring_parity(k, C::PB * NSUB), err,
+                         kErrWaitMma))
+            break;
+        }
         tc_fence_after_sync();
         const uint32_t a = tmem + static_cast<uint32_t>(C::TMEM_A + (j & 1) * 64);
         const uint64_t xd = xdesc0 + static_cast<uint64_t>(((i % C::XS) * C::X_BYTES) >> 4);
@@ -247,8 +257,6 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         c[u] = *reinterpret_cast<const uint4*>(qrow + (((4 + u) ^ (r & 7)) << 4));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qempty[qs]);
       // A buffer (j & 1) was last read by the items of slab j - 2.
       bool free_a = true;
       if (j >= 2) {
@@ -262,10 +270,13 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_after_sync();
       const uint32_t ta = t_lane + static_cast<uint32_t>(C::TMEM_A + (j & 1) * 64);
       tmem_st32x32(ta, o);
-      // tcgen05.st takes its source registers when it issues, so they can be
-      // refilled with the second half.
+      tmem_st_wait();  // the source registers are refilled below
 #pragma unroll
       for (int u = 0; u < 4; ++u) expand16(c[u], o + 8 * u);
+      // The codes have been consumed (shared-memory loads complete): the
+      // slab's q slot may be refilled.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qempty[qs]);
       tmem_st32x32(ta + 32u, o);
       tmem_st_wait();
       tc_fence_before_sync();
@@ -283,7 +294,6 @@ __global__ void __launch_bounds__(512, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
         const int m0 = (tile % mtiles) * (BT * NSUB), n0 = (tile / mtiles) * 128;
-        const int n = n0 + quad * 32 + lane;
         const float* sw_row = sw + static_cast<int64_t>(n0 >> 7) * KB;
         uint64_t acc[BT / 2];
 #pragma unroll
@@ -317,20 +327,38 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&pempty[i % C::PB]);
+          if (lane == 0) mbar_arrive(&pempty[(i % C::PB) * NSUB + t]);
         }
+        if (!ok) break;
+        // Output: the warp holds y[mt .. mt + BT)[n0 + 32q .. + 32) with one
+        // weight row (column of y) per lane. Sixteen tokens at a time go
+        // through shared memory as rows of 32 BF16, so that each lane then
+        // stores 16 contiguous values (32 bytes) of one row of y.
         const int mt = m0 + t * BT;
-        if (ok && n < N && mt < M) {
-          uint16_t* ycol = reinterpret_cast<uint16_t*>(y) + n;
-          const int mcount = min(BT, M - mt);
+        const int nw = n0 + quad * 32;  // first column of this warp
+        uint8_t* stg = sOut + (warp - 8) * C::OUT_BYTES;
+        const int rr = lane >> 1, hh = lane & 1;  // row and half this lane stores
 #pragma unroll
-          for (int e = 0; e < BT / 2; ++e) {
-            const uint32_t b2 = cvt_bf16x2_pair(acc[e]);
-            if (2 * e < mcount)
-              ycol[static_cast<int64_t>(mt + 2 * e) * ldy] = static_cast<uint16_t>(b2 & 0xFFFFu);
-            if (2 * e + 1 < mcount)
-              ycol[static_cast<int64_t>(mt + 2 * e + 1) * ldy] = static_cast<uint16_t>(b2 >> 16);
+        for (int g = 0; g < BT / 16; ++g) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t b2 = cvt_bf16x2_pair(acc[8 * g + e]);
+            *reinterpret_cast<uint16_t*>(stg + (2 * e) * 64 + lane * 2) = static_cast<uint16_t>(b2 & 0xFFFFu);
+            *reinterpret_cast<uint16_t*>(stg + (2 * e + 1) * 64 + lane * 2) = static_cast<uint16_t>(b2 >> 16);
           }
+          __syncwarp();
+          const uint8_t* src = stg + rr * 64 + hh * 32;
+          const int m = mt + 16 * g + rr, c0 = nw + 16 * hh;
+          if (m < M && c0 < N) {
+            uint16_t* dst = reinterpret_cast<uint16_t*>(y) + static_cast<int64_t>(m) * ldy + c0;
+            if (c0 + 16 <= N) {
+              reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(src)[0];
+              reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(src)[1];
+            } else {
+              for (int c = 0; c < N - c0; ++c) dst[c] = reinterpret_cast<const uint16_t*>(src)[c];
+            }
+          }
+          __syncwarp();  // the next group overwrites the buffer
         }
       }
     }

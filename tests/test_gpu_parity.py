@@ -256,3 +256,24 @@ def test_repeat_calls_are_deterministic():
         a = bf16_bits(f(x_d, q_d, s_d))
         b = bf16_bits(f(x_d, q_d, s_d))
         assert np.array_equal(a, b)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", ["w8a16", "w8a8"])
+def test_large_repeat_calls_are_deterministic(mode):
+    """Many tiles per CTA, so every ring in the persistent GEMMs wraps many
+    times: six calls must give bit-identical outputs (a ring-reuse race shows
+    up as a sub-tile or a band of weight rows differing between calls)."""
+    M, K, N = 4096, 5120, 25600
+    g = torch.Generator(device="cpu").manual_seed(7)
+    w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16).to(DEV)
+    q_d, s_d = fb.quantize_weight(w)
+    f = fb.linear_w8a16 if mode == "w8a16" else fb.linear_w8a8
+    first = f(x, q_d, s_d)
+    out = torch.empty_like(first)
+    for _ in range(5):
+        f(x, q_d, s_d, out=out)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), first.view(torch.int16))
+    assert fb.read_device_error() == 0
