@@ -134,7 +134,8 @@ __global__ void __launch_bounds__(512, 1)
     for (int s = 0; s < C::XS; ++s) mbar_init(&xfull[s], 1);
     for (int b = 0; b < 2; ++b) mbar_init(&afull[b], 4);
     for (int b = 0; b < C::RD; ++b) mbar_init(&done[b], 1);
-    for (int b = 0; b < C::PB * NSUB; ++b) mbar_init(&pempty[b], 4);
+    // NSUB == 2: all eight epilogue warps promote every item.
+    for (int b = 0; b < C::PB * NSUB; ++b) mbar_init(&pempty[b], NSUB == 2 ? 8 : 4);
     mbar_init_fence();
   }
   if (warp == 2) {
@@ -285,7 +286,83 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else {
     setmaxnreg_inc<184>();
-    if (((warp - 8) >> 2) < NSUB) {
+    if constexpr (NSUB == 2) {
+      // ------------------------------------ promotion/epilogue (two sub-tiles)
+      // All eight warps promote every item: warp 8 + 4h + q owns TMEM lane
+      // quadrant q and token columns [64h, 64h + 64) of each item's partial,
+      // so a partial is read by eight warps at once (two 32-column loads
+      // each) and its slot is released sooner.
+      const int ew = warp - 8, quad = warp & 3, h = ew >> 2;
+      const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::TMEM_P +
+                              static_cast<uint32_t>(64 * h);
+      uint8_t* stg = sOut + ew * C::OUT_BYTES;
+      const int rr = lane >> 1, hh = lane & 1;  // row and half this lane stores
+      int j = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
+        const int m0 = (tile % mtiles) * (BT * NSUB), n0 = (tile / mtiles) * 128;
+        const float* sw_row = sw + static_cast<int64_t>(n0 >> 7) * KB;
+        uint64_t acc[64];  // acc[32t + p]: tokens 128t + 64h + 2p and 2p + 1
+#pragma unroll
+        for (int e = 0; e < 64; ++e) acc[e] = 0ull;
+        float s_next = __ldg(sw_row);
+        for (int kb = 0; kb < KB && ok; ++kb, ++j) {
+          const float s = s_next;
+          if (kb + 1 < KB) s_next = __ldg(sw_row + kb + 1);
+          const uint64_t s2 = pack_f32x2(s, s);
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int i = 2 * j + t;
+            if (!mbar_wait_warp(&done[i % C::RD], ring_parity(i, C::RD), err, kErrWaitEpilogue)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            const uint32_t tp = t_lane + static_cast<uint32_t>((i % C::PB) * BT);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              uint32_t p[32];
+              tmem_ld32x32(tp + 32u * c, p);
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                ffma2(acc[32 * t + 16 * c + e], pack_u32x2(p[2 * e], p[2 * e + 1]), s2);
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[(i % C::PB) * 2 + t]);
+          }
+        }
+        if (!ok) break;
+        // Output: sixteen tokens at a time through shared memory as rows of
+        // 32 BF16 (this warp's columns of y), then 32-byte stores per lane.
+        const int nw = n0 + quad * 32;  // first column of this warp
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t b2 = cvt_bf16x2_pair(acc[32 * t + 8 * g + e]);
+              *reinterpret_cast<uint16_t*>(stg + (2 * e) * 64 + lane * 2) = static_cast<uint16_t>(b2 & 0xFFFFu);
+              *reinterpret_cast<uint16_t*>(stg + (2 * e + 1) * 64 + lane * 2) = static_cast<uint16_t>(b2 >> 16);
+            }
+            __syncwarp();
+            const uint8_t* src = stg + rr * 64 + hh * 32;
+            const int m = m0 + 128 * t + 64 * h + 16 * g + rr, c0 = nw + 16 * hh;
+            if (m < M && c0 < N) {
+              uint16_t* dst = reinterpret_cast<uint16_t*>(y) + static_cast<int64_t>(m) * ldy + c0;
+              if (c0 + 16 <= N) {
+                reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(src)[0];
+                reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(src)[1];
+              } else {
+                for (int c = 0; c < N - c0; ++c) dst[c] = reinterpret_cast<const uint16_t*>(src)[c];
+              }
+            }
+            __syncwarp();  // the next group overwrites the buffer
+          }
+        }
+      }
+    } else if (((warp - 8) >> 2) < NSUB) {
       // ------------------------------------------------ promotion/epilogue
       const int t = (warp - 8) >> 2;  // token sub-tile
       const int quad = warp & 3;
