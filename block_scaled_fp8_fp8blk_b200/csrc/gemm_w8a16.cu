@@ -98,12 +98,50 @@ __device__ __forceinline__ uint32_t ring_parity(int item, int depth) {
   return static_cast<uint32_t>((item / depth) & 1);
 }
 
+// The slabs one CTA runs, as a run of segments (tile, [kb0, kb1)): whole
+// tiles blockIdx.x, + gridDim.x, ... (round robin), or with stream-K the
+// contiguous range [c U / G, (c + 1) U / G) of the U = tiles x KB slabs in
+// tile-major order (c = blockIdx.x, G = gridDim.x), which gives every CTA the
+// same number of slabs within one. Under stream-K a tile may be split across
+// consecutive CTAs; only a CTA's first and last segments can be partial.
+struct Schedule {
+  int64_t u, end, first;
+  int tile, KB, ntiles;
+  bool streamk;
+  __device__ Schedule(bool sk, int kb_per_tile, int tiles)
+      : tile(static_cast<int>(blockIdx.x)), KB(kb_per_tile), ntiles(tiles), streamk(sk) {
+    const int64_t U = static_cast<int64_t>(tiles) * kb_per_tile;
+    first = u = U * blockIdx.x / gridDim.x;
+    end = U * (blockIdx.x + 1) / gridDim.x;
+  }
+  __device__ int slabs() const {
+    if (streamk) return static_cast<int>(end - first);
+    return tile < ntiles ? ((ntiles - 1 - tile) / static_cast<int>(gridDim.x) + 1) * KB : 0;
+  }
+  __device__ bool next(int& t, int& kb0, int& kb1) {
+    if (streamk) {
+      if (u >= end) return false;
+      t = static_cast<int>(u / KB);
+      kb0 = static_cast<int>(u - static_cast<int64_t>(t) * KB);
+      kb1 = static_cast<int>(min(static_cast<int64_t>(KB), kb0 + (end - u)));
+      u += kb1 - kb0;
+      return true;
+    }
+    if (tile >= ntiles) return false;
+    t = tile;
+    kb0 = 0;
+    kb1 = KB;
+    tile += static_cast<int>(gridDim.x);
+    return true;
+  }
+};
+
 template <int BT, int NSUB>
 __global__ void __launch_bounds__(512, 1)
     w8a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_x,
                       const float* __restrict__ sw, __nv_bfloat16* __restrict__ y, int64_t ldy,
-                      int M, int N, int KB, int mtiles, int ntiles_total,
-                      unsigned* __restrict__ err) {
+                      int M, int N, int KB, int mtiles, int ntiles_total, int streamk,
+                      float* __restrict__ part, unsigned* __restrict__ err) {
   using C = W8A16Cfg<BT, NSUB>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
@@ -121,10 +159,7 @@ __global__ void __launch_bounds__(512, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + C::PB * NSUB);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Slabs this CTA will run: KB per tile, tiles blockIdx.x, +gridDim.x, ...
-  const int my_tiles =
-      static_cast<int>(blockIdx.x) < ntiles_total ? (ntiles_total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const int total_slabs = my_tiles * KB;
+  const int total_slabs = Schedule(streamk != 0, KB, ntiles_total).slabs();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::QS; ++s) {
@@ -157,9 +192,11 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_map(&tm_q);
       int j = 0;  // slab counter (across tiles)
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
+      Schedule sc(streamk != 0, KB, ntiles_total);
+      int tile, kb0, kb1;
+      while (ok && sc.next(tile, kb0, kb1)) {
         const int n0 = (tile / mtiles) * 128;
-        for (int kb = 0; kb < KB; ++kb, ++j) {
+        for (int kb = kb0; kb < kb1; ++kb, ++j) {
           const int qs = j % C::QS;
           if (!mbar_wait_sleepy(&qempty[qs], ring_parity(j, C::QS) ^ 1u, err, kErrWaitLoad)) {
             ok = false;
@@ -177,9 +214,11 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_map(&tm_x);
       int i = 0;  // item counter (across tiles)
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
+      Schedule sc(streamk != 0, KB, ntiles_total);
+      int tile, kb0, kb1;
+      while (ok && sc.next(tile, kb0, kb1)) {
         const int m0 = (tile % mtiles) * (BT * NSUB);
-        for (int kb = 0; kb < KB && ok; ++kb) {
+        for (int kb = kb0; kb < kb1 && ok; ++kb) {
           for (int t = 0; t < NSUB; ++t, ++i) {
             const int xs = i % C::XS;
             if (i >= C::XS) {  // the item that last used this slot has finished
@@ -369,16 +408,19 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::TMEM_P;
       int j = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
+      Schedule sc(streamk != 0, KB, ntiles_total);
+      int tile, kb0, kb1;
+      bool first_segment = true;
+      while (ok && sc.next(tile, kb0, kb1)) {
         const int m0 = (tile % mtiles) * (BT * NSUB), n0 = (tile / mtiles) * 128;
         const float* sw_row = sw + static_cast<int64_t>(n0 >> 7) * KB;
         uint64_t acc[BT / 2];
 #pragma unroll
         for (int e = 0; e < BT / 2; ++e) acc[e] = 0ull;
-        float s_next = __ldg(sw_row);
-        for (int kb = 0; kb < KB; ++kb, ++j) {
+        float s_next = __ldg(sw_row + kb0);
+        for (int kb = kb0; kb < kb1; ++kb, ++j) {
           const float s = s_next;
-          if (kb + 1 < KB) s_next = __ldg(sw_row + kb + 1);
+          if (kb + 1 < kb1) s_next = __ldg(sw_row + kb + 1);
           const int i = j * NSUB + t;
           if (!mbar_wait_warp(&done[i % C::RD], ring_parity(i, C::RD), err, kErrWaitEpilogue)) {
             ok = false;
@@ -407,6 +449,23 @@ __global__ void __launch_bounds__(512, 1)
           if (lane == 0) mbar_arrive(&pempty[(i % C::PB) * NSUB + t]);
         }
         if (!ok) break;
+        const bool whole = kb0 == 0 && kb1 == KB;
+        const int slot = first_segment ? 0 : 1;
+        first_segment = false;
+        if (!whole) {
+          // Part of a tile split across CTAs (stream-K): the FP32 partial goes
+          // to slot (CTA, first or last segment) of the workspace, [BT][128]
+          // with the weight row fastest; w8a16_streamk_reduce adds the slots.
+          float* dst = part + (static_cast<int64_t>(blockIdx.x) * 2 + slot) * (BT * 128) + quad * 32 + lane;
+#pragma unroll
+          for (int e = 0; e < BT / 2; ++e) {
+            float lo, hi;
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc[e]));
+            dst[(2 * e) * 128] = lo;
+            dst[(2 * e + 1) * 128] = hi;
+          }
+          continue;
+        }
         // Output: the warp holds y[mt .. mt + BT)[n0 + 32q .. + 32) with one
         // weight row (column of y) per lane. Sixteen tokens at a time go
         // through shared memory as rows of 32 BF16, so that each lane then
@@ -450,10 +509,41 @@ __global__ void __launch_bounds__(512, 1)
   }
 }
 
+// Stream-K fix-up: y for every tile whose slabs were split across CTAs, the
+// sum of the CTAs' FP32 partials in slab order (CTA c holds slabs
+// [c U / G, (c + 1) U / G)), rounded once to BF16. One CTA per tile and
+// token, one thread per weight row; tiles run by a single CTA were written
+// directly.
+template <int BT>
+__global__ void __launch_bounds__(128) w8a16_streamk_reduce(const float* __restrict__ part,
+                                                            uint16_t* __restrict__ y, int64_t ldy,
+                                                            int, int N, int KB, int ntiles, int G) {
+  const int tile = blockIdx.x, m = blockIdx.y, r = threadIdx.x;
+  const int64_t U = static_cast<int64_t>(ntiles) * KB;
+  // CTA whose range holds slab x: the largest c with c U / G <= x.
+  auto owner = [&](int64_t x) { return static_cast<int>(((x + 1) * G - 1) / U); };
+  const int c_first = owner(static_cast<int64_t>(tile) * KB);
+  const int c_last = owner(static_cast<int64_t>(tile + 1) * KB - 1);
+  if (c_first == c_last) return;
+  // The tile is c_first's last segment (slot 1) unless c_first starts in it.
+  const bool first_starts_here = U * c_first / G == static_cast<int64_t>(tile) * KB;
+  const int n = tile * 128 + r;
+  if (n >= N) return;
+  float acc = 0.0f;
+  for (int c = c_first; c <= c_last; ++c) {
+    const int slot = (c == c_first && !first_starts_here) ? 1 : 0;
+    acc += part[(static_cast<int64_t>(c) * 2 + slot) * (BT * 128) + m * 128 + r];
+  }
+  y[static_cast<int64_t>(m) * ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+}
+
+// CTAs a stream-K launch may use (the workspace is sized for this many).
+constexpr int kStreamKMaxCtas = 160;
+
 template <int BT, int NSUB>
 cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                       int64_t ldq, const float* sw, uint16_t* y, int64_t ldy, int64_t M,
-                      int64_t N, int64_t K) {
+                      int64_t N, int64_t K, void* ws, size_t ws_bytes) {
   using C = W8A16Cfg<BT, NSUB>;
   CUtensorMap tq, tx;
   if (!make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, N, ldq, 128, 128))
@@ -473,26 +563,48 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
   const int64_t mtiles = cdiv(M, BT * NSUB), tiles = mtiles * cdiv(N, 128);
   // Slab and item counters are 32-bit per CTA.
   if (tiles * cdiv(K, 128) * NSUB > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  const int grid = static_cast<int>(tiles < L.num_sms ? tiles : L.num_sms);
-  kern<<<grid, C::THREADS, C::SMEM, L.stream>>>(
+  // One token tile (M <= 128): stream-K over the slabs, so every SM streams
+  // the same share of the weights however few 128-row tiles there are.
+  const int64_t KB = cdiv(K, 128);
+  const bool streamk = NSUB == 1;
+  int64_t grid = streamk ? tiles * KB : tiles;
+  const int64_t cap = streamk ? (L.num_sms < kStreamKMaxCtas ? L.num_sms : kStreamKMaxCtas) : L.num_sms;
+  if (grid > cap) grid = cap;
+  if (streamk && (!ws || ws_bytes < static_cast<size_t>(grid) * 2 * BT * 128 * sizeof(float)))
+    return cudaErrorInvalidValue;
+  kern<<<static_cast<int>(grid), C::THREADS, C::SMEM, L.stream>>>(
       tq, tx, sw, reinterpret_cast<__nv_bfloat16*>(y), ldy, static_cast<int>(M),
-      static_cast<int>(N), static_cast<int>(cdiv(K, 128)), static_cast<int>(mtiles),
-      static_cast<int>(tiles), L.err);
+      static_cast<int>(N), static_cast<int>(KB), static_cast<int>(mtiles),
+      static_cast<int>(tiles), streamk ? 1 : 0, static_cast<float*>(ws), L.err);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !streamk) return e;
+  w8a16_streamk_reduce<BT><<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(M < BT ? M : BT)),
+                             128, 0, L.stream>>>(
+      static_cast<const float*>(ws), y, ldy, static_cast<int>(M), static_cast<int>(N),
+      static_cast<int>(KB), static_cast<int>(tiles), static_cast<int>(grid));
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t w8a16_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+namespace {
+int token_tile(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
+}  // namespace
+
+// M <= 128 runs stream-K: FP32 partials of split tiles, two slots per CTA.
+size_t w8a16_workspace_bytes(int64_t M, int64_t, int64_t) {
+  if (M > 128) return 0;
+  return static_cast<size_t>(kStreamKMaxCtas) * 2 * token_tile(M) * 128 * sizeof(float);
+}
 
 cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                               int64_t ldq, const float* sw, uint16_t* y, int64_t ldy, int64_t M,
-                              int64_t N, int64_t K, void*, size_t) {
-  if (M <= 16) return launch_bt<16, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
-  if (M <= 32) return launch_bt<32, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
-  if (M <= 64) return launch_bt<64, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
-  if (M <= 128) return launch_bt<128, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
-  return launch_bt<128, 2>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K);
+                              int64_t N, int64_t K, void* ws, size_t ws_bytes) {
+  if (M <= 16) return launch_bt<16, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
+  if (M <= 32) return launch_bt<32, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
+  if (M <= 64) return launch_bt<64, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
+  if (M <= 128) return launch_bt<128, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
+  return launch_bt<128, 2>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
 }
 
 }  // namespace fp8blk

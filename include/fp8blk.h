@@ -124,7 +124,10 @@ FP8BLK_EXPORT fp8blk_status fp8blk_quantize_act(const void* x, int64_t M, int64_
  *   y : BF16 [M][ldy], ldy >= N, ldy % 8 == 0; must not alias the inputs (output)
  *   workspace : fp8blk_workspace_size(0, M, N, K) bytes, 256-byte aligned
  *               (may be NULL when that size is 0); its contents on entry do
- *               not matter and are scratch on return.
+ *               not matter and are scratch on return. For M <= 128 the slabs
+ *               are split evenly over the SMs (stream-K) and the workspace
+ *               holds the FP32 partials of tiles split between SMs (at most
+ *               160 x 2 x 128 x 128 x 4 bytes); for M > 128 it is 0 bytes.
  * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED_DEVICE, WORKSPACE, CUDA.
  * ------------------------------------------------------------------------- */
 FP8BLK_EXPORT fp8blk_status fp8blk_linear_w8a16(const void* x, int64_t ldx, const uint8_t* q, int64_t ldq,
