@@ -16,7 +16,8 @@ import os
 
 __all__ = [
     "Fp8BlkError", "lib", "quantize_weight", "dequantize", "quantize_act", "linear_w8a16",
-    "linear_w8a8", "workspace_size", "encode_e4m3", "read_device_error", "version",
+    "linear_w8a8", "linear_w8a8_quantized", "workspace_size", "encode_e4m3", "read_device_error",
+    "version",
     "LIB_PATH", "EXPORTS",
 ]
 
@@ -40,6 +41,7 @@ EXPORTS = {
     "fp8blk_linear_w8a16": (_st, [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]),
     "fp8blk_linear_w8a8": (_st, [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]),
     "fp8blk_linear_w8a8_noalloc": (_st, [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p]),
+    "fp8blk_linear_w8a8_quantized": (_st, [_p, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p]),
     "fp8blk_workspace_size": (_sz, [_int, _i64, _i64, _i64]),
     "fp8blk_encode_e4m3": (_st, [_p, _i64, _p, _p]),
     "fp8blk_read_device_error": (_st, [ctypes.POINTER(ctypes.c_uint32)]),
@@ -173,6 +175,21 @@ def linear_w8a16(x, q, scale_inv, out=None, workspace=None):
 def linear_w8a8(x, q, scale_inv, out=None, workspace=None):
     """y = x . dequant(q, scale_inv)^T with x quantized per 1x128 K-group to E4M3."""
     return _linear(1, "fp8blk_linear_w8a8", x, q, scale_inv, out, workspace)
+
+
+def linear_w8a8_quantized(qx, sx, q, scale_inv, M=None, out=None):
+    """W8A8 linear on (qx, sx) from quantize_act; M defaults to qx.shape[0]."""
+    import torch
+    M = qx.shape[0] if M is None else M
+    K = qx.shape[1]
+    N = q.shape[0]
+    if out is None:
+        out = _padded(M, N, _round_up(max(N, 1), 8), torch.bfloat16, qx.device)
+    _check(lib().fp8blk_linear_w8a8_quantized(qx.data_ptr(), _ld(qx), sx.data_ptr(), sx.stride(0),
+                                              q.data_ptr(), _ld(q), scale_inv.data_ptr(),
+                                              out.data_ptr(), _ld(out), M, N, K, _stream()),
+           "fp8blk_linear_w8a8_quantized")
+    return out
 
 
 def encode_e4m3(v):

@@ -253,6 +253,33 @@ fp8blk_status fp8blk_linear_w8a8(const void* x, int64_t ldx, const uint8_t* q, i
                                       static_cast<uint16_t*>(y), ldy, M, N, K));
 }
 
+fp8blk_status fp8blk_linear_w8a8_quantized(const uint8_t* qx, int64_t ldqx, const float* sx,
+                                           int64_t ldsx, const uint8_t* q, int64_t ldq,
+                                           const float* scale_inv, void* y, int64_t ldy, int64_t M,
+                                           int64_t N, int64_t K, fp8blk_stream stream) {
+  if (M < 0 || N < 0 || K < 0) return FP8BLK_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP8BLK_OK;
+  if (!y || ldy < N) return FP8BLK_ERR_INVALID_ARG;
+  if (ldy % 8 || !aligned(y, 16)) return FP8BLK_ERR_ALIGNMENT;
+  if (K > 0) {
+    if (!qx || !sx || !q || !scale_inv || ldqx < K || ldsx < M || ldq < K)
+      return FP8BLK_ERR_INVALID_ARG;
+    if (M > kInt32Max || N > kInt32Max || K > kInt32Max) return FP8BLK_ERR_INVALID_ARG;
+    if (ldqx % 16 || ldq % 16 || !aligned(qx, 16) || !aligned(q, 16) || !aligned(sx, 4) ||
+        !aligned(scale_inv, 4))
+      return FP8BLK_ERR_ALIGNMENT;
+  }
+  Launch L;
+  fp8blk_status st = make_launch(stream, &L);
+  if (st != FP8BLK_OK) return st;
+  if (K == 0)  // empty sum: y = 0
+    return cuda_status(cudaMemset2DAsync(y, static_cast<size_t>(ldy) * 2, 0,
+                                         static_cast<size_t>(N) * 2, static_cast<size_t>(M),
+                                         L.stream));
+  return cuda_status(launch_w8a8_gemm(L, qx, ldqx, sx, ldsx, q, ldq, scale_inv,
+                                      static_cast<uint16_t*>(y), ldy, M, N, K));
+}
+
 size_t fp8blk_workspace_size(int mode, int64_t M, int64_t N, int64_t K) {
   if (M < 0 || N < 0 || K < 0) return 0;
   if (M == 0 || N == 0 || K == 0) return 0;

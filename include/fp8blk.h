@@ -182,6 +182,25 @@ FP8BLK_EXPORT fp8blk_status fp8blk_linear_w8a8_noalloc(const void* x, int64_t ld
                                                        int64_t ldy, int64_t M, int64_t N, int64_t K,
                                                        fp8blk_stream stream);
 
+/* ---------------------------------------------------------------------------
+ * W8A8 linear on activations already quantized by fp8blk_quantize_act, so
+ * that sibling linears reading the same x (Q, K and V; gate and up) quantize
+ * it once (FastVideo PR #1829, "Changes": the Blackwell route quantizes the
+ * activations before the groupwise GEMM). Computes
+ *   y[m][n] = BF16( sum_kb sx[kb][m] * s[n/128][kb] * P_kb[m][n] )
+ * exactly as fp8blk_linear_w8a8 does after its own quantization step.
+ *   qx : uint8 [M][ldqx], ldqx >= K, ldqx % 16 == 0, 16-byte aligned (input)
+ *   sx : float [ceil(K/128)][ldsx], ldsx >= M, 4-byte aligned          (input)
+ *   q, scale_inv, y, M, N, K : as for fp8blk_linear_w8a8.
+ * No workspace. Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA.
+ * ------------------------------------------------------------------------- */
+FP8BLK_EXPORT fp8blk_status fp8blk_linear_w8a8_quantized(const uint8_t* qx, int64_t ldqx,
+                                                         const float* sx, int64_t ldsx,
+                                                         const uint8_t* q, int64_t ldq,
+                                                         const float* scale_inv, void* y,
+                                                         int64_t ldy, int64_t M, int64_t N,
+                                                         int64_t K, fp8blk_stream stream);
+
 /* Workspace bytes for a linear: mode 0 = W8A16, 1 = W8A8. Pure host function;
  * returns 0 for an invalid mode or negative sizes. */
 FP8BLK_EXPORT size_t fp8blk_workspace_size(int mode, int64_t M, int64_t N, int64_t K);

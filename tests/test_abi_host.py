@@ -124,6 +124,25 @@ def test_linear_validation(lib, name):
         assert call(ws=P + 16) == 4   # workspace must be 256-byte aligned
 
 
+def test_linear_w8a8_quantized_validation(lib):
+    f = lib.fp8blk_linear_w8a8_quantized
+    M, N, K = 64, 384, 256
+    ok = [P, K, P, M, P, K, P, P, N, M, N, K, None]
+
+    def call(**kw):
+        a = list(ok)
+        idx = dict(qx=0, ldqx=1, sx=2, ldsx=3, q=4, ldq=5, s=6, y=7, ldy=8, M=9, N=10, K=11)
+        for k, v in kw.items():
+            a[idx[k]] = v
+        return f(*a)
+
+    assert call(M=-1) == 1 and call(K=-1) == 1
+    assert call(M=0) == 0 and call(N=0) == 0
+    assert call(qx=None) == 1 and call(sx=None) == 1 and call(q=None) == 1 and call(y=None) == 1
+    assert call(ldqx=K - 16) == 1 and call(ldsx=M - 1) == 1 and call(ldq=K - 16) == 1
+    assert call(ldqx=K + 8) == 2 and call(qx=PM) == 2 and call(sx=P + 2) == 2 and call(y=PM) == 2
+
+
 def test_encode_validation(lib):
     f = lib.fp8blk_encode_e4m3
     assert f(P, -1, P, None) == 1

@@ -277,3 +277,17 @@ def test_large_repeat_calls_are_deterministic(mode):
         torch.cuda.synchronize()
         assert torch.equal(out.view(torch.int16), first.view(torch.int16))
     assert fb.read_device_error() == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [W.RAGGED, W.Workload("m300_k640_n512", 300, 640, 512)], ids=lambda w: w.name)
+def test_linear_w8a8_quantized_matches_linear_w8a8(wl):
+    """Quantizing the activations once (fp8blk_quantize_act) and running the
+    GEMM on them gives exactly what fp8blk_linear_w8a8 gives."""
+    wb, q, s = weight_case(wl)
+    x_d = to_dev_bf16(synth.bf16_bits(wl.x_bf16()), -(-wl.K // 8) * 8)
+    q_d, s_d = to_dev_u8(q), torch.from_numpy(s).to(DEV)
+    ref = bf16_bits(fb.linear_w8a8(x_d, q_d, s_d))
+    qx, sx = fb.quantize_act(x_d)
+    got = bf16_bits(fb.linear_w8a8_quantized(qx, sx, q_d, s_d))
+    assert np.array_equal(got, ref)
