@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--workload", default="linear_m512_k5120_n25600")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-ab", action="store_true",
+                    help="skip the A/B timings of the library BF16 route and shared act quantization")
     return ap.parse_args()
 
 
@@ -369,6 +371,49 @@ def main():
                        "d2h_bytes_per_step": 2 * 2 * M * N}
     else:
         line["e2e"] = None
+
+    # A/B, outside the step: (1) the route of FP8-less tensor cores, our
+    # dequantize then a library BF16 GEMM on the expanded weight, against the
+    # fused W8A16 call; (2) one activation quantization shared by sibling
+    # linears (fp8blk_quantize_act + fp8blk_linear_w8a8_quantized) against
+    # the all-in-one W8A8 call, which re-quantizes x each time.
+    if not args.no_ab:
+        def timed(fn, iters=20):
+            ts = []
+            for _ in range(iters):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(); fn(); b.record()
+                ts.append((a, b))
+            torch.cuda.synchronize()
+            return 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ts)
+
+        y_lib = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        qx, sx = fb.quantize_act(x)
+        for _ in range(3):
+            fb.dequantize(q, s, out=wd); torch.matmul(x, wd.t(), out=y_lib)
+            fb.linear_w8a8_quantized(qx, sx, q, s, out=y8)
+        torch.cuda.synchronize()
+        us_deq = timed(lambda: fb.dequantize(q, s, out=wd))
+        us_mm = timed(lambda: torch.matmul(x, wd.t(), out=y_lib))
+        us_route = timed(lambda: (fb.dequantize(q, s, out=wd), torch.matmul(x, wd.t(), out=y_lib)))
+        us_w16 = timed(lambda: fb.linear_w8a16(x, q, s, out=y16, workspace=ws16))
+        us_act = timed(lambda: fb.quantize_act(x, qx, sx))
+        us_w8q = timed(lambda: fb.linear_w8a8_quantized(qx, sx, q, s, out=y8))
+        us_w8 = timed(lambda: fb.linear_w8a8(x, q, s, out=y8, workspace=ws8))
+        fl = 2.0 * M * N * K
+        line["ab"] = {
+            "library_bf16_route": {
+                "dequantize_us": us_deq, "cublas_bf16_matmul_us": us_mm,
+                "route_us": us_route, "route_tflops": fl / (us_route * 1e-6) / 1e12,
+                "linear_w8a16_us": us_w16, "linear_w8a16_tflops": fl / (us_w16 * 1e-6) / 1e12,
+                "speedup_w8a16_over_route": us_route / us_w16},
+            "shared_act_quantization": {
+                "quantize_act_us": us_act, "linear_w8a8_quantized_us": us_w8q,
+                "linear_w8a8_us": us_w8,
+                "saved_per_sibling_us": us_w8 - us_w8q},
+            "iters": 20, "l2": "flushed before each timed call"}
+        del y_lib, qx, sx
 
     assert fb.read_device_error() == 0
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
