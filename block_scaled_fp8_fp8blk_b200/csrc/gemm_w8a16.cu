@@ -26,14 +26,17 @@
 // Warp roles (16 warps; registers rebalanced per warpgroup with setmaxnreg):
 //   warp 0       TMA producer of weight-code slabs [128 x 128 B] (q ring);
 //   warp 1       TMA producer of activation sub-tiles [BT x 128 BF16] (x ring);
-//   warps 2..    MMA issuers, one per sub-tile t: per slab 8 x (M=128, N=BT,
+//   warps 2, 3   MMA issuers of alternate items: per item 8 x (M=128, N=BT,
 //                K=16), A from TMEM, B from shared memory, into a ring of TMEM
 //                partials shared in item order (warp 2 also allocates TMEM);
 //   warps 4-7    expansion: one weight row per thread (TMEM lane), 128 codes
-//                -> 64 bf16x2 words -> tcgen05.st into one of two A buffers;
-//   warps 8-15   promotion/epilogue: warp (8 + 4t + q) owns TMEM lanes of
-//                quadrant q for sub-tile t: acc[BT] += P * s with packed
-//                FP32x2 FMAs, then BF16 stores of y (coalesced along n).
+//                -> 64 bf16x2 words -> tcgen05.st into one of AB A buffers
+//                (with one sub-tile, of the even slabs only);
+//   warps 8-15   two sub-tiles: promotion/epilogue, acc += P * s with packed
+//                FP32x2 FMAs, then BF16 stores of y (coalesced along n);
+//                one sub-tile: warps 8-11 promote and store, warps 12-15
+//                expand the odd slabs (the conversion is the per-slab cost
+//                at small token counts, so two groups overlap it).
 // Every wait is bounded (kWaitLimitCycles) and reports to the error word.
 #include <cuda_bf16.h>
 
@@ -48,16 +51,22 @@ struct W8A16Cfg {
   static constexpr int Q_BYTES = 128 * 128;  // FP8 weight slab
   static constexpr int X_ATOM = BT * 128;    // BT rows x 64 BF16 (128 B)
   static constexpr int X_BYTES = 2 * X_ATOM; // one sub-tile slab
-  static constexpr int QS = BT >= 128 ? 3 : (BT >= 64 ? 4 : 7);
+  // With one sub-tile two warpgroups expand alternate slabs; the q ring is
+  // then even, so each q slot (and its barriers) belongs to one of them.
+  static constexpr int NEXP = NSUB == 1 ? 2 : 1;
+  static constexpr int QS = NSUB == 2 ? 3 : (BT >= 64 ? 4 : 8);
   static constexpr int XS = BT >= 128 ? (NSUB == 2 ? 5 : 4) : (BT >= 64 ? 6 : 7);
   static constexpr int THREADS = 512;
   static constexpr int PB = 3;                  // TMEM partial ring depth (items)
   static constexpr int RD = 8;                  // "group done" barrier ring depth (items)
-  static constexpr int TMEM_A = 0;              // 2 buffers x 64 columns
-  static constexpr int TMEM_P = 128;            // PB buffers x BT columns
+  // Expanded-weight (A) buffers in TMEM, 64 columns each; with one sub-tile
+  // the two issuers take alternate slabs, each over AB / 2 of them.
+  static constexpr int AB = (NSUB == 1 && BT <= 64) ? 4 : 2;
+  static constexpr int TMEM_A = 0;              // AB buffers x 64 columns
+  static constexpr int TMEM_P = 64 * AB;        // PB buffers x BT columns
   static constexpr int TMEM_USED = TMEM_P + PB * BT;
   static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
-  static constexpr int NBAR = 2 * QS + XS + 2 + RD + PB * NSUB;
+  static constexpr int NBAR = 2 * QS + XS + AB + RD + PB * 2;
   static constexpr int OUT_BYTES = 16 * 64;     // per epilogue warp: 16 tokens x 32 BF16
   static constexpr size_t SMEM_TILES = static_cast<size_t>(QS) * Q_BYTES +
                                        static_cast<size_t>(XS) * X_BYTES + 4 * NSUB * OUT_BYTES;
@@ -71,7 +80,10 @@ struct W8A16Cfg {
   // barrier waits on it before item i + RD can be committed. The activation
   // producer recycles an x slot XS items later (RD >= XS keeps the loads of
   // item i + RD behind its wait on item i). The expansion waits for the items
-  // of slab j - 2 before filling slab j's A buffer. The promotion warps of
+  // of slab j - AB before filling slab j's A buffer (RD >= AB * NSUB puts
+  // item i + RD in that slab or a later one; with two expansion groups the
+  // items a group waits on have one parity, and so do the items of one
+  // "done" barrier, RD being even). The promotion warps of
   // sub-tile t release a partial after waiting on its item; partials are used
   // in item order across both issuers, so item k waits for the promotion of
   // item k - PB, and with PB = 3 and two issuers each issuer waits on the
@@ -79,7 +91,15 @@ struct W8A16Cfg {
   // (i + RD) / NSUB, whose expansion waited for both items of an earlier
   // slab, one of which waited for the promotion of an item of sub-tile t at
   // or after i (checked for RD = 8, PB = 3, NSUB <= 2).
-  static_assert(RD >= XS && RD >= 2 * NSUB && RD - PB >= NSUB - 1, "done ring depth");
+  static_assert(RD >= XS && RD >= AB * NSUB && RD - PB >= NSUB - 1, "done ring depth");
+  // Two issuers own alternate items (item i: issuer i % 2). The x slot of
+  // item i last held item i - XS; the issuer of item i has already waited
+  // on the promotion of item i - 5 (at its previous item), so item i - XS
+  // has been issued and its load waited on whenever XS is even (same
+  // issuer) or odd and at least 5 (the other issuer, which issues in order).
+  static_assert(XS % 2 == 0 || XS >= 5, "x ring depth with two issuers");
+  static_assert(AB % 2 == 0 && RD % 2 == 0, "rings shared by alternating issuers");
+  static_assert(NEXP == 1 || QS % NEXP == 0, "q ring shared by alternating expansion groups");
 };
 
 // Expand 16 E4M3 codes (one 16-byte chunk) into 8 bf16x2 words.
@@ -136,6 +156,62 @@ struct Schedule {
   }
 };
 
+// ------------------------------------------------------------------ expansion
+// One warpgroup expands the slabs j = eg, eg + NEXP, ... of its CTA: thread r
+// (TMEM lane r) turns weight row r's 128 codes into 64 bf16x2 words and
+// stores them with tcgen05.st into A buffer j % AB.
+template <class C, int NSUB>
+__device__ __forceinline__ void expand_slabs(int eg, int total_slabs, const uint8_t* sQ,
+                                             uint32_t tmem, uint64_t* qfull, uint64_t* qempty,
+                                             uint64_t* afull, uint64_t* done, unsigned* err) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quad = warp & 3;
+  const int r = quad * 32 + lane;  // weight row within the tile == TMEM lane
+  const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+  for (int j = eg; j < total_slabs; j += C::NEXP) {
+    const int qs = j % C::QS;
+    if (!mbar_wait_warp(&qfull[qs], ring_parity(j, C::QS), err, kErrWaitExpand)) break;
+    // Row r of the 128-byte-swizzled slab: 16-byte chunk c sits at chunk
+    // position c ^ (r & 7).
+    const uint8_t* qrow = sQ + qs * C::Q_BYTES + r * 128;
+    uint4 c[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      c[u] = *reinterpret_cast<const uint4*>(qrow + ((u ^ (r & 7)) << 4));
+    uint32_t o[32];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) expand16(c[u], o + 8 * u);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      c[u] = *reinterpret_cast<const uint4*>(qrow + (((4 + u) ^ (r & 7)) << 4));
+    // A buffer j % AB was last read by the items of slab j - AB.
+    bool free_a = true;
+    if (j >= C::AB) {
+#pragma unroll
+      for (int t = 0; t < NSUB; ++t) {
+        const int ia = NSUB * (j - C::AB) + t;
+        free_a = free_a && mbar_wait_warp(&done[ia % C::RD], ring_parity(ia, C::RD), err, kErrWaitExpand);
+      }
+    }
+    if (!free_a) break;
+    tc_fence_after_sync();
+    const uint32_t ta = t_lane + static_cast<uint32_t>(C::TMEM_A + (j % C::AB) * 64);
+    tmem_st32x32(ta, o);
+    tmem_st_wait();  // the source registers are refilled below
+#pragma unroll
+    for (int u = 0; u < 4; ++u) expand16(c[u], o + 8 * u);
+    // The codes have been consumed (shared-memory loads complete): the
+    // slab's q slot may be refilled.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&qempty[qs]);
+    tmem_st32x32(ta + 32u, o);
+    tmem_st_wait();
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&afull[j % C::AB]);
+  }
+}
+
 template <int BT, int NSUB>
 __global__ void __launch_bounds__(512, 1)
     w8a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_x,
@@ -154,9 +230,9 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* qempty = qfull + C::QS;    // codes read            (4 expansion warps)
   uint64_t* xfull = qempty + C::QS;    // x sub-tile landed     (1 arrival + tx)
   uint64_t* afull = xfull + C::XS;     // A buffer written      (4 expansion warps)
-  uint64_t* done = afull + 2;          // group's MMAs complete (1 commit)
-  uint64_t* pempty = done + C::RD;     // partial consumed      (4 epilogue warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + C::PB * NSUB);
+  uint64_t* done = afull + C::AB;      // item's MMAs complete  (1 commit)
+  uint64_t* pempty = done + C::RD;     // partial consumed      (4 or 8 epilogue warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + C::PB * 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total_slabs = Schedule(streamk != 0, KB, ntiles_total).slabs();
@@ -167,10 +243,11 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&qempty[s], 4);
     }
     for (int s = 0; s < C::XS; ++s) mbar_init(&xfull[s], 1);
-    for (int b = 0; b < 2; ++b) mbar_init(&afull[b], 4);
+    for (int b = 0; b < C::AB; ++b) mbar_init(&afull[b], 4);
     for (int b = 0; b < C::RD; ++b) mbar_init(&done[b], 1);
-    // NSUB == 2: all eight epilogue warps promote every item.
-    for (int b = 0; b < C::PB * NSUB; ++b) mbar_init(&pempty[b], NSUB == 2 ? 8 : 4);
+    // One barrier per (partial slot, issuer). NSUB == 2: all eight epilogue
+    // warps promote every item.
+    for (int b = 0; b < C::PB * 2; ++b) mbar_init(&pempty[b], NSUB == 2 ? 8 : 4);
     mbar_init_fence();
   }
   if (warp == 2) {
@@ -181,6 +258,8 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // The stream-K fix-up kernel may be scheduled now; it waits for this grid.
+  if (streamk) pdl_launch_dependents();
 
   // Each warpgroup sets its register budget at the top of its role:
   // 128 x (56 + 80 + 184 + 184) = 64512 of the 65536 the block holds.
@@ -237,31 +316,32 @@ __global__ void __launch_bounds__(512, 1)
       }
       for (int s = 0; s < C::XS && s < i; ++s)
         mbar_wait(&xfull[s], last_parity((i - s + C::XS - 1) / C::XS), err, kErrWaitLoad);
-    } else if (warp >= 2 && warp < 2 + NSUB && lane == 0) {
+    } else if (warp >= 2 && warp < 4 && lane == 0) {
       // ------------------------------------------------------- MMA issuers
-      // Issuer t runs the items of sub-tile t; with two issuers one's waits
-      // and commits hide behind the other's MMAs. Descriptors are formed
-      // once; stepping through shared memory adds (bytes >> 4) to their
+      // Issuer u runs the items i with i % 2 == u: sub-tile u of every slab
+      // (NSUB == 2), or every other slab (NSUB == 1). One issuer's waits and
+      // commits hide behind the other's MMAs. Descriptors are formed once;
+      // stepping through shared memory adds (bytes >> 4) to their
       // start-address field.
-      const int t = warp - 2;
+      const int u = warp - 2;
       const uint64_t xdesc0 = sw128_kmajor_desc(smem_addr(sX));
       int last = -1;
-      for (int j = 0; j < total_slabs; ++j) {
-        const int i = j * NSUB + t;
-        if (!mbar_wait(&afull[j & 1], ring_parity(j, 2), err, kErrWaitMma)) break;
+      for (int j = NSUB == 1 ? u : 0; j < total_slabs; j += NSUB == 1 ? 2 : 1) {
+        const int i = NSUB == 1 ? j : 2 * j + u;
+        if (!mbar_wait(&afull[j % C::AB], ring_parity(j, C::AB), err, kErrWaitMma)) break;
         if (!mbar_wait(&xfull[i % C::XS], ring_parity(i, C::XS), err, kErrWaitMma)) break;
         // Partial slot i % PB last held item k = i - PB, whose promotion
-        // arrives on that slot's barrier for k's sub-tile. Each issuer meets
+        // arrives on that slot's barrier for k's issuer. Each issuer meets
         // every phase of the barriers it waits on, in order (a parity wait
         // cannot tell a phase from the one two before or after).
         if (i >= C::PB) {
           const int k = i - C::PB;
-          if (!mbar_wait(&pempty[(k % C::PB) * NSUB + k % NSUB], ring_parity(k, C::PB * NSUB), err,
+          if (!mbar_wait(&pempty[(k % C::PB) * 2 + (k & 1)], ring_parity(k, C::PB * 2), err,
                          kErrWaitMma))
             break;
         }
         tc_fence_after_sync();
-        const uint32_t a = tmem + static_cast<uint32_t>(C::TMEM_A + (j & 1) * 64);
+        const uint32_t a = tmem + static_cast<uint32_t>(C::TMEM_A + (j % C::AB) * 64);
         const uint64_t xd = xdesc0 + static_cast<uint64_t>(((i % C::XS) * C::X_BYTES) >> 4);
         const uint32_t d = tmem + static_cast<uint32_t>(C::TMEM_P + (i % C::PB) * BT);
 #pragma unroll
@@ -276,53 +356,8 @@ __global__ void __launch_bounds__(512, 1)
       if (last >= 0) mbar_wait(&done[last % C::RD], ring_parity(last, C::RD), err, kErrWaitMma);
     }
   } else if (wg == 1) {
-    // ---------------------------------------------------------- expansion
     setmaxnreg_dec<80>();
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // weight row within the tile == TMEM lane
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    for (int j = 0; j < total_slabs; ++j) {
-      const int qs = j % C::QS;
-      if (!mbar_wait_warp(&qfull[qs], ring_parity(j, C::QS), err, kErrWaitExpand)) break;
-      // Row r of the 128-byte-swizzled slab: 16-byte chunk c sits at chunk
-      // position c ^ (r & 7).
-      const uint8_t* qrow = sQ + qs * C::Q_BYTES + r * 128;
-      uint4 c[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        c[u] = *reinterpret_cast<const uint4*>(qrow + ((u ^ (r & 7)) << 4));
-      uint32_t o[32];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) expand16(c[u], o + 8 * u);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        c[u] = *reinterpret_cast<const uint4*>(qrow + (((4 + u) ^ (r & 7)) << 4));
-      // A buffer (j & 1) was last read by the items of slab j - 2.
-      bool free_a = true;
-      if (j >= 2) {
-#pragma unroll
-        for (int t = 0; t < NSUB; ++t) {
-          const int ia = NSUB * (j - 2) + t;
-          free_a = free_a && mbar_wait_warp(&done[ia % C::RD], ring_parity(ia, C::RD), err, kErrWaitExpand);
-        }
-      }
-      if (!free_a) break;
-      tc_fence_after_sync();
-      const uint32_t ta = t_lane + static_cast<uint32_t>(C::TMEM_A + (j & 1) * 64);
-      tmem_st32x32(ta, o);
-      tmem_st_wait();  // the source registers are refilled below
-#pragma unroll
-      for (int u = 0; u < 4; ++u) expand16(c[u], o + 8 * u);
-      // The codes have been consumed (shared-memory loads complete): the
-      // slab's q slot may be refilled.
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qempty[qs]);
-      tmem_st32x32(ta + 32u, o);
-      tmem_st_wait();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[j & 1]);
-    }
+    expand_slabs<C, NSUB>(0, total_slabs, sQ, tmem, qfull, qempty, afull, done, err);
   } else {
     setmaxnreg_inc<184>();
     if constexpr (NSUB == 2) {
@@ -446,7 +481,7 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&pempty[(i % C::PB) * NSUB + t]);
+          if (lane == 0) mbar_arrive(&pempty[(i % C::PB) * 2 + (i & 1)]);
         }
         if (!ok) break;
         const bool whole = kb0 == 0 && kb1 == KB;
@@ -455,7 +490,7 @@ __global__ void __launch_bounds__(512, 1)
         if (!whole) {
           // Part of a tile split across CTAs (stream-K): the FP32 partial goes
           // to slot (CTA, first or last segment) of the workspace, [BT][128]
-          // with the weight row fastest; w8a16_streamk_reduce adds the slots.
+          // with the weight row fastest; w8a16_streamk_fixup adds the slots.
           float* dst = part + (static_cast<int64_t>(blockIdx.x) * 2 + slot) * (BT * 128) + quad * 32 + lane;
 #pragma unroll
           for (int e = 0; e < BT / 2; ++e) {
@@ -497,6 +532,9 @@ __global__ void __launch_bounds__(512, 1)
           __syncwarp();  // the next group overwrites the buffer
         }
       }
+    } else {
+      // One sub-tile: warps 12-15 are the second expansion group (odd slabs).
+      expand_slabs<C, NSUB>(1, total_slabs, sQ, tmem, qfull, qempty, afull, done, err);
     }
   }
 
@@ -509,36 +547,81 @@ __global__ void __launch_bounds__(512, 1)
   }
 }
 
-// Stream-K fix-up: y for every tile whose slabs were split across CTAs, the
-// sum of the CTAs' FP32 partials in slab order (CTA c holds slabs
-// [c U / G, (c + 1) U / G)), rounded once to BF16. One CTA per tile and
-// token, one thread per weight row; tiles run by a single CTA were written
-// directly.
-template <int BT>
-__global__ void __launch_bounds__(128) w8a16_streamk_reduce(const float* __restrict__ part,
-                                                            uint16_t* __restrict__ y, int64_t ldy,
-                                                            int, int N, int KB, int ntiles, int G) {
-  const int tile = blockIdx.x, m = blockIdx.y, r = threadIdx.x;
-  const int64_t U = static_cast<int64_t>(ntiles) * KB;
-  // CTA whose range holds slab x: the largest c with c U / G <= x.
-  auto owner = [&](int64_t x) { return static_cast<int>(((x + 1) * G - 1) / U); };
-  const int c_first = owner(static_cast<int64_t>(tile) * KB);
-  const int c_last = owner(static_cast<int64_t>(tile + 1) * KB - 1);
-  if (c_first == c_last) return;
-  // The tile is c_first's last segment (slot 1) unless c_first starts in it.
-  const bool first_starts_here = U * c_first / G == static_cast<int64_t>(tile) * KB;
-  const int n = tile * 128 + r;
-  if (n >= N) return;
-  float acc = 0.0f;
-  for (int c = c_first; c <= c_last; ++c) {
-    const int slot = (c == c_first && !first_starts_here) ? 1 : 0;
-    acc += part[(static_cast<int64_t>(c) * 2 + slot) * (BT * 128) + m * 128 + r];
-  }
-  y[static_cast<int64_t>(m) * ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
-}
-
 // CTAs a stream-K launch may use (the workspace is sized for this many).
 constexpr int kStreamKMaxCtas = 160;
+
+// The tiles a stream-K launch splits across CTAs, worked out on the host:
+// CTA c holds slabs [c U / G, (c + 1) U / G) of the U = tiles x KB slabs, so
+// a tile is split when a range boundary falls inside it. Each split tile
+// lists its first contributor c0 (whose last segment it is), the number of
+// contributors, and the workspace slot c0 wrote (0 if the tile was also
+// c0's first segment, else 1); later contributors wrote slot 0.
+struct SplitTiles {
+  int count;
+  int tile[kStreamKMaxCtas];
+  short c0[kStreamKMaxCtas];
+  unsigned char ncontrib[kStreamKMaxCtas];
+  unsigned char slot0[kStreamKMaxCtas];
+};
+
+SplitTiles split_tiles(int64_t ntiles, int64_t KB, int64_t G) {
+  SplitTiles st{};
+  const int64_t U = ntiles * KB;
+  for (int64_t c0 = 0; c0 + 1 < G; ++c0) {
+    const int64_t x = U * (c0 + 1) / G;  // first slab of CTA c0 + 1
+    const int64_t t = x / KB, s0 = t * KB;
+    const int64_t c0_start = U * c0 / G;
+    if (x == s0 || c0_start > s0) continue;  // no split here, or not the tile's first boundary
+    const int64_t c1 = ((s0 + KB) * G - 1) / U;  // holds the tile's last slab
+    st.tile[st.count] = static_cast<int>(t);
+    st.c0[st.count] = static_cast<short>(c0);
+    st.ncontrib[st.count] = static_cast<unsigned char>(c1 - c0 + 1);
+    st.slot0[st.count] = static_cast<unsigned char>(c0_start == s0 ? 0 : 1);
+    ++st.count;
+  }
+  return st;
+}
+
+// Stream-K fix-up: y of every split tile, the sum of its contributors' FP32
+// partials in slab order, rounded once to BF16. Block (i, g) handles split
+// tile i for tokens [8 g, 8 g + 8) with one thread per weight row and token
+// parity, every partial load issued before the sums. Tiles run by a single
+// CTA were written directly. Launched as a programmatic dependent of the
+// GEMM: it waits for the GEMM grid to complete before it reads a partial.
+template <int BT>
+__global__ void __launch_bounds__(256) w8a16_streamk_fixup(const __grid_constant__ SplitTiles st,
+                                                           const float* __restrict__ part,
+                                                           uint16_t* __restrict__ y, int64_t ldy,
+                                                           int M, int N) {
+  pdl_wait();
+  const int i = static_cast<int>(blockIdx.x);
+  const int r = threadIdx.x & 127;
+  const int n = st.tile[i] * 128 + r;
+  if (n >= N) return;
+  const int c0 = st.c0[i], nc = st.ncontrib[i], slot0 = st.slot0[i];
+  const int mbase = static_cast<int>(blockIdx.y) * 8 + (threadIdx.x >> 7);
+  float acc[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) acc[u] = 0.0f;
+  for (int c = 0; c < nc; ++c) {
+    const float* p = part + (static_cast<int64_t>(c0 + c) * 2 + (c == 0 ? slot0 : 0)) * (BT * 128) + r;
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int m = mbase + 2 * u;
+      v[u] = m < M && m < BT ? p[m * 128] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] += v[u];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int m = mbase + 2 * u;
+    if (m < M && m < BT)
+      y[static_cast<int64_t>(m) * ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[u]));
+  }
+}
+
 
 template <int BT, int NSUB>
 cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
@@ -554,11 +637,16 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
   {
-    // The setmaxnreg split (64512 registers) needs 128 per thread at launch.
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kern));
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs * C::THREADS < 128 * (56 + 80 + 184 + 184)) return cudaErrorInvalidConfiguration;
+    // The setmaxnreg split (64512 registers) needs 128 per thread at launch
+    // (checked once per kernel).
+    static const cudaError_t regs = [&] {
+      cudaFuncAttributes fa;
+      cudaError_t r = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kern));
+      if (r != cudaSuccess) return r;
+      return fa.numRegs * C::THREADS < 128 * (56 + 80 + 184 + 184) ? cudaErrorInvalidConfiguration
+                                                                   : cudaSuccess;
+    }();
+    if (regs != cudaSuccess) return regs;
   }
   const int64_t mtiles = cdiv(M, BT * NSUB), tiles = mtiles * cdiv(N, 128);
   // Slab and item counters are 32-bit per CTA.
@@ -577,12 +665,22 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
       static_cast<int>(N), static_cast<int>(KB), static_cast<int>(mtiles),
       static_cast<int>(tiles), streamk ? 1 : 0, static_cast<float*>(ws), L.err);
   e = cudaGetLastError();
-  if (e != cudaSuccess || !streamk) return e;
-  w8a16_streamk_reduce<BT><<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(M < BT ? M : BT)),
-                             128, 0, L.stream>>>(
-      static_cast<const float*>(ws), y, ldy, static_cast<int>(M), static_cast<int>(N),
-      static_cast<int>(KB), static_cast<int>(tiles), static_cast<int>(grid));
-  return cudaGetLastError();
+  if (e != cudaSuccess || !streamk || grid < 2) return e;
+  const SplitTiles st = split_tiles(tiles, KB, grid);
+  if (st.count == 0) return cudaSuccess;
+  const int mt = static_cast<int>(M < BT ? M : BT);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(st.count), static_cast<unsigned>((mt + 7) / 8));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, w8a16_streamk_fixup<BT>, st, static_cast<const float*>(ws), y,
+                            ldy, static_cast<int>(M), static_cast<int>(N));
 }
 
 }  // namespace

@@ -107,6 +107,14 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, u
   return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
+// Programmatic dependent launch (sm_90 and later): let the kernel launched
+// after this one in the stream be scheduled now, and, in that kernel, wait
+// until the kernel before it has completed with its memory visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Position in a ring of mbarrier-guarded slots: slot index and the parity of
 // the phase that slot is on.
 struct Ring {
