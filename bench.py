@@ -9,7 +9,8 @@ on the headline layer (M=512 tokens, K=5120, N=25600, the largest linear of a
 `value` = FLOPs of the step's two linears (2 * 2MNK) / device time of the
 step, summed over ranks / max over ranks. Per-call times, TFLOP/s, weight
 GB/s and roofline fractions are reported beside it. L2 is flushed between
-steps (a 512 MiB memset outside the step's CUDA events).
+steps outside the step's CUDA events: a 512 MiB memset, then a 256 MiB read,
+so the step starts with no input in L2 and no dirty flush lines to write back.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle on a bounded sample
@@ -37,6 +38,7 @@ METRIC = "block-FP8 linear TFLOP/s and weight-stream GB/s (M=512,K=5120,N=25600)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
 FLUSH_BYTES = 512 << 20
+FLUSH_READ_BYTES = 256 << 20
 
 
 def parse():
@@ -244,6 +246,14 @@ def main():
     ws16 = torch.empty(max(1, fb.workspace_size(0, M, N, K)), dtype=torch.uint8, device=dev)
     ws8 = torch.empty(max(1, fb.workspace_size(1, M, N, K)), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def flush_l2():
+        # Write more than L2 holds, then read another buffer twice its size:
+        # the step starts with an L2 that holds none of its inputs and no
+        # dirty lines of the flush to write back.
+        flush.zero_()
+        flush_rd.sum()
 
     def step(ev=None):
         if ev: ev[0].record()
@@ -257,7 +267,7 @@ def main():
         if ev: ev[4].record()
 
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush_l2()
         step()
     torch.cuda.synchronize()
     assert fb.read_device_error() == 0
@@ -270,7 +280,7 @@ def main():
     clocks.start()
     time.sleep(0.15)
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         step(events[i])
     torch.cuda.synchronize()
     barrier()
@@ -331,7 +341,7 @@ def main():
         "dtype": "e4m3/bf16 operands, f32 accumulate", "data": "synthetic",
         "config": {"workload": wl.name, "M": M, "K": K, "N": N,
                    "step": "quantize_weight + dequantize + linear_w8a16 + linear_w8a8",
-                   "l2": "flushed between steps (512 MiB memset outside the step events)",
+                   "l2": "flushed between steps outside the step events (512 MiB memset, then a 256 MiB read so no dirty flush lines remain)",
                    "parallelism": f"replicas x{world}"},
         "weight_stream_gbs": {c: call_stats[c]["weight_stream_gbs"]
                               for c in ("linear_w8a16", "linear_w8a8")},
@@ -381,7 +391,7 @@ def main():
         def timed(fn, iters=20):
             ts = []
             for _ in range(iters):
-                flush.zero_()
+                flush_l2()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(); fn(); b.record()
                 ts.append((a, b))
@@ -412,7 +422,7 @@ def main():
                 "quantize_act_us": us_act, "linear_w8a8_quantized_us": us_w8q,
                 "linear_w8a8_us": us_w8,
                 "saved_per_sibling_us": us_w8 - us_w8q},
-            "iters": 20, "l2": "flushed before each timed call"}
+            "iters": 20, "l2": "flushed (memset + read) before each timed call"}
         del y_lib, qx, sx
 
     assert fb.read_device_error() == 0
