@@ -246,7 +246,7 @@ def main():
     ws16 = torch.empty(max(1, fb.workspace_size(0, M, N, K)), dtype=torch.uint8, device=dev)
     ws8 = torch.empty(max(1, fb.workspace_size(1, M, N, K)), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flush_rd = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_rd = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.float32, device=dev)
 
     def flush_l2():
         # Write more than L2 holds, then read another buffer twice its size:

@@ -250,7 +250,7 @@ fp8blk_status fp8blk_linear_w8a8(const void* x, int64_t ldx, const uint8_t* q, i
       launch_quantize_act(L, static_cast<const uint16_t*>(x), M, K, ldx, qx, ldqx, sx, ldsx);
   if (e != cudaSuccess) return FP8BLK_ERR_CUDA;
   return cuda_status(launch_w8a8_gemm(L, qx, ldqx, sx, ldsx, q, ldq, scale_inv,
-                                      static_cast<uint16_t*>(y), ldy, M, N, K));
+                                      static_cast<uint16_t*>(y), ldy, M, N, K, true));
 }
 
 fp8blk_status fp8blk_linear_w8a8_quantized(const uint8_t* qx, int64_t ldqx, const float* sx,
@@ -277,7 +277,7 @@ fp8blk_status fp8blk_linear_w8a8_quantized(const uint8_t* qx, int64_t ldqx, cons
                                          static_cast<size_t>(N) * 2, static_cast<size_t>(M),
                                          L.stream));
   return cuda_status(launch_w8a8_gemm(L, qx, ldqx, sx, ldsx, q, ldq, scale_inv,
-                                      static_cast<uint16_t*>(y), ldy, M, N, K));
+                                      static_cast<uint16_t*>(y), ldy, M, N, K, false));
 }
 
 size_t fp8blk_workspace_size(int mode, int64_t M, int64_t N, int64_t K) {

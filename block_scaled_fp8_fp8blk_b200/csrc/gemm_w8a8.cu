@@ -130,6 +130,10 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
       const uint32_t bytes = is_a ? C::A_BYTES : C::B_BYTES;
       uint8_t* dst0 = smem + (is_a ? 0 : C::A_BYTES);
       tma_prefetch_map(map);
+      // Launched as a programmatic dependent of the activation quantizer:
+      // the weights may stream at once, the activation codes only once that
+      // kernel has completed (a no-op for an ordinary launch).
+      if (is_a) pdl_wait();
       int j = 0;  // slab counter (across tiles)
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
@@ -177,6 +181,7 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
   } else {
     setmaxnreg_inc<C::REG_EPI>();
     // -------------------------------------------------- promotion/epilogue
+    pdl_wait();  // the activation scales come from the kernel before
     const int ew = warp - 4;
     const int quad = warp & 3;  // TMEM lanes this warp may access
     const int h = ew >> 2;      // partial columns [128h, 128h + 128)
@@ -267,7 +272,8 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
 
 cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, const float* sx,
                              int64_t ldsx, const uint8_t* q, int64_t ldq, const float* sw,
-                             uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K) {
+                             uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                             bool after_act_quant) {
   using C = W8A8Cfg;
   CUtensorMap ta, tb, ty;
   if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, K, M, ldqx, 128, C::BM))
@@ -286,21 +292,36 @@ cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, c
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
   {
-    // The register split needs the launch allocation it was sized for.
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kern));
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs < C::REG_LAUNCH) return cudaErrorInvalidConfiguration;
+    // The register split needs the launch allocation it was sized for
+    // (checked once).
+    static const cudaError_t regs = [&] {
+      cudaFuncAttributes fa;
+      cudaError_t r = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kern));
+      if (r != cudaSuccess) return r;
+      return fa.numRegs < C::REG_LAUNCH ? cudaErrorInvalidConfiguration : cudaSuccess;
+    }();
+    if (regs != cudaSuccess) return regs;
   }
   const int64_t mtiles = cdiv(M, C::BM), tiles = mtiles * cdiv(N, C::BN);
   // Slab counters are 32-bit per CTA.
   if (tiles * cdiv(K, 128) > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   const int grid = static_cast<int>(tiles < L.num_sms ? tiles : L.num_sms);
-  kern<<<grid, C::THREADS, C::SMEM, L.stream>>>(
-      ta, tb, ty, sx, ldsx, sw, y, ldy, static_cast<int>(M), static_cast<int>(N),
-      static_cast<int>(n_tma), static_cast<int>(cdiv(K, 128)), static_cast<int>(mtiles),
-      static_cast<int>(tiles), L.err);
-  return cudaGetLastError();
+  // After the activation quantizer: a programmatic dependent launch, so the
+  // GEMM's set-up and weight loads overlap that kernel.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_act_quant ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, sx, ldsx, sw, y, ldy, static_cast<int>(M),
+                            static_cast<int>(N), static_cast<int>(n_tma),
+                            static_cast<int>(cdiv(K, 128)), static_cast<int>(mtiles),
+                            static_cast<int>(tiles), L.err);
 }
 
 }  // namespace fp8blk

@@ -26,9 +26,12 @@ cudaError_t launch_quantize_act(const Launch& L, const uint16_t* x, int64_t M, i
                                 int64_t ldx, uint8_t* qx, int64_t ldqx, float* sx, int64_t ldsx);
 cudaError_t launch_encode_e4m3(const Launch& L, const float* v, int64_t n, uint8_t* codes);
 
+// after_act_quant: launched right after launch_quantize_act on the same
+// stream, as its programmatic dependent (weight loads overlap that kernel).
 cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, const float* sx,
                              int64_t ldsx, const uint8_t* q, int64_t ldq, const float* scale_inv,
-                             uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K);
+                             uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                             bool after_act_quant);
 
 size_t w8a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,

@@ -99,7 +99,7 @@ extern "C" fp8blk_status fp8blk_linear_w8a8_noalloc(const void* x, int64_t ldx, 
       cudaSuccess)
     return FP8BLK_ERR_CUDA;
   return launch_w8a8_gemm(L, qx, ldqx, sx, ldsx, q, ldq, scale_inv, static_cast<uint16_t*>(y), ldy,
-                          M, N, K) == cudaSuccess
+                          M, N, K, true) == cudaSuccess
              ? FP8BLK_OK
              : FP8BLK_ERR_CUDA;
 }

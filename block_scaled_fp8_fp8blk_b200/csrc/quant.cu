@@ -292,6 +292,9 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
                                                            uint8_t* __restrict__ qx, int64_t ldqx,
                                                            float* __restrict__ sx, int64_t ldsx,
                                                            int KB) {
+  // The W8A8 GEMM launched after this kernel may be scheduled now: it reads
+  // the codes and scales only after griddepcontrol.wait.
+  pdl_launch_dependents();
   const int j = threadIdx.x & 15;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * 16 + (threadIdx.x >> 4);
   const bool live = g < M * KB;
