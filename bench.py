@@ -50,6 +50,12 @@ def parse():
     ap.add_argument("--workload", default="linear_m512_k5120_n25600")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--stack", type=int, default=0,
+                    help="instead of the step: stream the FP8 weights of this many 32B-shaped "
+                         "layers from pinned host memory (one GPU)")
+    ap.add_argument("--stack-mode", type=int, default=0, choices=[0, 1], help="0 W8A16, 1 W8A8")
+    ap.add_argument("--stack-m", type=int, default=512)
+    ap.add_argument("--stack-slots", type=int, default=2)
     ap.add_argument("--no-ab", action="store_true",
                     help="skip the A/B timings of the library BF16 route and shared act quantization")
     return ap.parse_args()
@@ -202,10 +208,120 @@ def traffic_for(kernel_file: str, key: str):
     return None
 
 
+# Linears of one decoder layer of the 32B class the pages' encoder belongs to
+# (hidden 5120, 64 query heads x 128, 8 KV heads, MLP 25600): (K, N).
+STACK_LAYER = [("qkv", 5120, 10240), ("o_proj", 8192, 5120), ("gate_up", 5120, 51200),
+               ("down", 25600, 5120)]
+
+
+def stack_arm(args):
+    """Layerwise FP8 weight streaming: every layer's codes and scales in their
+    own pinned host buffers, run through a ring of device slots
+    (fp8blk_streamed_linears), against the same linears on resident weights
+    and against the copies alone. One GPU; synthetic codes (no NaN)."""
+    import torch
+    import block_scaled_fp8_fp8blk_b200 as fb
+    L, M, mode, nslots = args.stack, args.stack_m, args.stack_mode, args.stack_slots
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(5)
+    host, dev_w, xs, ys = [], [], {}, {}
+    slot_bytes, ws_need, layer_bytes = 0, 0, 0
+    for name, K, N in STACK_LAYER:
+        ldq = -(-K // 16) * 16
+        slot_bytes = max(slot_bytes, fb.stream_slot_bytes(N, K, ldq))
+        ws_need = max(ws_need, fb.workspace_size(mode, M, N, K))
+        layer_bytes += N * ldq + 4 * (-(-N // 128)) * (-(-K // 128))
+        xs[name] = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+        ys[name] = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    slot_bytes = -(-slot_bytes // 256) * 256
+    for layer in range(L):
+        for name, K, N in STACK_LAYER:
+            ldq = -(-K // 16) * 16
+            # codes 0x00..0x7E with a random sign: every finite E4M3 value
+            q = (torch.randint(0, 0x7F, (N, ldq), device=dev, generator=g, dtype=torch.uint8)
+                 | (torch.randint(0, 2, (N, ldq), device=dev, generator=g, dtype=torch.uint8) << 7))
+            s = torch.rand(-(-N // 128), -(-K // 128), device=dev, generator=g) * 1e-3 + 1e-4
+            qh = torch.empty((N, ldq), dtype=torch.uint8, pin_memory=True)
+            qh.copy_(q)
+            sh = torch.empty(s.shape, dtype=torch.float32, pin_memory=True)
+            sh.copy_(s)
+            host.append((name, qh[:, :K], sh))
+            dev_w.append((q[:, :K], s))
+    torch.cuda.synchronize()
+    jobs = [(mode, qh, sh, xs[name], ys[name]) for name, qh, sh in host]
+    slots = torch.empty(nslots * slot_bytes, dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(1, ws_need), dtype=torch.uint8, device=dev)
+    compute, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    events = [torch.cuda.Event() for _ in range(2 * nslots)]
+    f = fb.linear_w8a16 if mode == 0 else fb.linear_w8a8
+
+    def timed(run, reps):
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(compute)
+            copy.wait_event(a)
+            run()
+            compute.wait_stream(copy)
+            b.record(compute)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ts)
+
+    def streamed():
+        fb.streamed_linears(jobs, slots, slot_bytes, nslots, ws, compute, copy, events)
+
+    def resident():
+        with torch.cuda.stream(compute):
+            for (name, qh, sh), (q, s) in zip(host, dev_w):
+                f(xs[name], q, s, out=ys[name], workspace=ws)
+
+    def copies_only():
+        with torch.cuda.stream(copy):
+            for i, (name, qh, sh) in enumerate(host):
+                k = i % nslots
+                slots[k * slot_bytes:k * slot_bytes + qh.shape[0] * qh.stride(0)].copy_(
+                    qh.as_strided((qh.shape[0] * qh.stride(0),), (1,)), non_blocking=True)
+
+    reps = max(3, min(args.steps, 10))
+    for run in (streamed, resident, copies_only):
+        timed(run, 1)
+    t_stream = timed(streamed, reps) / L
+    t_res = timed(resident, reps) / L
+    t_copy = timed(copies_only, reps) / L
+    assert fb.read_device_error() == 0
+    h2d = layer_bytes / (t_stream * 1e-3) / 1e9
+    line = {
+        "metric": "streamed FP8 linear stack: ms per layer, weights from pinned host memory",
+        "value": t_stream, "unit": "ms/layer", "higher_is_better": False, "n_gpus": 1,
+        "steps": reps, "data": "synthetic (random finite E4M3 codes and scales)",
+        "dtype": "e4m3 weights, bf16 activations" if mode == 0 else "e4m3 weights and activations",
+        "config": {"workload": f"stack32b_m{M}_L{L}", "layers": L, "linears_per_layer": 4,
+                   "shapes_KN": [[k, n] for _, k, n in STACK_LAYER], "M": M,
+                   "mode": "w8a16" if mode == 0 else "w8a8", "slots": nslots},
+        "fp8_bytes_per_layer": layer_bytes,
+        "h2d_gbs_streamed": h2d,
+        "copy_only_ms_per_layer": t_copy,
+        "h2d_gbs_copy_only": layer_bytes / (t_copy * 1e-3) / 1e9,
+        "resident_ms_per_layer": t_res,
+        "overlap_efficiency": max(t_copy, t_res) / t_stream,
+        "device_weight_bytes_streamed": nslots * slot_bytes,
+        "device_weight_bytes_resident_fp8": L * layer_bytes,
+        "device_weight_bytes_resident_bf16": L * sum(2 * k * n for _, k, n in STACK_LAYER),
+        "bf16_stream_ms_per_layer_at_same_h2d": sum(2 * k * n for _, k, n in STACK_LAYER) / (h2d * 1e9) * 1e3,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     from block_scaled_fp8_fp8blk_b200 import workloads
     wl = workloads.ALL[args.workload]
+    if args.stack > 0:
+        if int(os.environ.get("RANK", "0")) == 0:
+            stack_arm(args)
+        return
     if args.impl == "reference":
         return reference_arm(args, wl)
 

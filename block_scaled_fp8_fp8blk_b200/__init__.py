@@ -17,7 +17,7 @@ import os
 __all__ = [
     "Fp8BlkError", "lib", "quantize_weight", "dequantize", "quantize_act", "linear_w8a16",
     "linear_w8a8", "linear_w8a8_quantized", "workspace_size", "encode_e4m3", "read_device_error",
-    "version",
+    "version", "LinearJob", "stream_slot_bytes", "streamed_linears",
     "LIB_PATH", "EXPORTS",
 ]
 
@@ -33,6 +33,14 @@ STATUS = {
 _i64, _p, _sz, _int = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
 _st = ctypes.c_int
 
+
+class LinearJob(ctypes.Structure):
+    """fp8blk_linear_job: one linear of a streamed sequence (host weights)."""
+    _fields_ = [("mode", ctypes.c_int32), ("q_host", _p), ("scale_host", _p), ("ldq", _i64),
+                ("x", _p), ("ldx", _i64), ("y", _p), ("ldy", _i64),
+                ("M", _i64), ("N", _i64), ("K", _i64)]
+
+
 # name -> (restype, argtypes), mirroring include/fp8blk.h
 EXPORTS = {
     "fp8blk_quantize_weight": (_st, [_p, _i64, _i64, _i64, _p, _i64, _p, _p]),
@@ -43,6 +51,9 @@ EXPORTS = {
     "fp8blk_linear_w8a8_noalloc": (_st, [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p]),
     "fp8blk_linear_w8a8_quantized": (_st, [_p, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p]),
     "fp8blk_workspace_size": (_sz, [_int, _i64, _i64, _i64]),
+    "fp8blk_stream_slot_bytes": (_sz, [_i64, _i64, _i64]),
+    "fp8blk_streamed_linears": (_st, [ctypes.POINTER(LinearJob), _i64, _p, _sz, ctypes.c_int32,
+                                      _p, _sz, _p, _p, ctypes.POINTER(_p)]),
     "fp8blk_encode_e4m3": (_st, [_p, _i64, _p, _p]),
     "fp8blk_read_device_error": (_st, [ctypes.POINTER(ctypes.c_uint32)]),
     "fp8blk_status_string": (ctypes.c_char_p, [_int]),
@@ -190,6 +201,40 @@ def linear_w8a8_quantized(qx, sx, q, scale_inv, M=None, out=None):
                                               out.data_ptr(), _ld(out), M, N, K, _stream()),
            "fp8blk_linear_w8a8_quantized")
     return out
+
+
+def stream_slot_bytes(N: int, K: int, ldq: int) -> int:
+    return lib().fp8blk_stream_slot_bytes(N, K, ldq)
+
+
+def streamed_linears(jobs, slots, slot_bytes: int, nslots: int, workspace, compute, copy, events):
+    """Run linears whose weights are in (pinned) host memory through nslots
+    device weight slots (fp8blk_streamed_linears).
+
+    jobs: list of (mode, q_host, s_host, x, y) with mode 0 = W8A16, 1 = W8A8,
+    q_host uint8 [N, K] / s_host float32 (CPU tensors, pinned for overlap;
+    q_host's row stride is ldq), x BF16 [M, K] and y BF16 [M, N] on the GPU.
+    slots: uint8 CUDA tensor of nslots * slot_bytes; compute / copy:
+    torch.cuda.Stream; events: 2 * nslots torch.cuda.Event (created here by
+    a first record on `compute` if they have no handle yet).
+    """
+    arr = (LinearJob * max(1, len(jobs)))()
+    for i, (mode, qh, sh, x, y) in enumerate(jobs):
+        M, K = x.shape
+        N = qh.shape[0]
+        if qh.shape[1] != K or y.shape != (M, N):
+            raise ValueError("job shapes disagree")
+        arr[i] = LinearJob(mode, qh.data_ptr(), sh.data_ptr(), _ld(qh), x.data_ptr(), _ld(x),
+                           y.data_ptr(), _ld(y), M, N, K)
+    for e in events:
+        if not e.cuda_event:
+            e.record(compute)
+    ev = (_p * max(1, len(events)))(*[e.cuda_event for e in events])
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().fp8blk_streamed_linears(arr, len(jobs), slots.data_ptr(), slot_bytes, nslots,
+                                         ws_ptr, ws_len, compute.cuda_stream, copy.cuda_stream, ev),
+           "fp8blk_streamed_linears")
 
 
 def encode_e4m3(v):

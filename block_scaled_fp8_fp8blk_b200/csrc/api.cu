@@ -127,6 +127,27 @@ cudaError_t ensure_smem_limit(const void* kernel, size_t bytes) {
   return e;
 }
 
+// The argument checks of the linear calls, without any CUDA call (also used
+// to check every job of a streamed sequence before anything is enqueued).
+fp8blk_status validate_linear(const void* x, int64_t ldx, const uint8_t* q, int64_t ldq,
+                              const float* scale_inv, const void* y, int64_t ldy, int64_t M,
+                              int64_t N, int64_t K, const void* ws, size_t ws_bytes,
+                              size_t ws_need) {
+  if (M < 0 || N < 0 || K < 0) return FP8BLK_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP8BLK_OK;
+  if (!y || ldy < N) return FP8BLK_ERR_INVALID_ARG;
+  if (ldy % 8 || !aligned(y, 16)) return FP8BLK_ERR_ALIGNMENT;
+  if (K > 0) {
+    if (!x || !q || !scale_inv || ldx < K || ldq < K) return FP8BLK_ERR_INVALID_ARG;
+    if (M > kInt32Max || N > kInt32Max || K > kInt32Max) return FP8BLK_ERR_INVALID_ARG;
+    if (ldx % 8 || ldq % 16 || !aligned(x, 16) || !aligned(q, 16) || !aligned(scale_inv, 4))
+      return FP8BLK_ERR_ALIGNMENT;
+    if (ws_need > 0 && (!ws || ws_bytes < ws_need || !aligned(ws, 256)))
+      return FP8BLK_ERR_WORKSPACE;
+  }
+  return FP8BLK_OK;
+}
+
 // The launch context of the current device (stream, error word, SM count),
 // for entry points defined in other files.
 fp8blk_status current_launch(fp8blk_stream stream, Launch* L) { return make_launch(stream, L); }
@@ -190,22 +211,13 @@ fp8blk_status check_linear(const void* x, int64_t ldx, const uint8_t* q, int64_t
                            int64_t K, void* ws, size_t ws_bytes, size_t ws_need,
                            fp8blk_stream stream, Launch* L, bool* done) {
   *done = false;
-  if (M < 0 || N < 0 || K < 0) return FP8BLK_ERR_INVALID_ARG;
+  fp8blk_status st = validate_linear(x, ldx, q, ldq, scale_inv, y, ldy, M, N, K, ws, ws_bytes, ws_need);
+  if (st != FP8BLK_OK) return st;
   if (M == 0 || N == 0) {
     *done = true;
     return FP8BLK_OK;
   }
-  if (!y || ldy < N) return FP8BLK_ERR_INVALID_ARG;
-  if (ldy % 8 || !aligned(y, 16)) return FP8BLK_ERR_ALIGNMENT;
-  if (K > 0) {
-    if (!x || !q || !scale_inv || ldx < K || ldq < K) return FP8BLK_ERR_INVALID_ARG;
-    if (M > kInt32Max || N > kInt32Max || K > kInt32Max) return FP8BLK_ERR_INVALID_ARG;
-    if (ldx % 8 || ldq % 16 || !aligned(x, 16) || !aligned(q, 16) || !aligned(scale_inv, 4))
-      return FP8BLK_ERR_ALIGNMENT;
-    if (ws_need > 0 && (!ws || ws_bytes < ws_need || !aligned(ws, 256)))
-      return FP8BLK_ERR_WORKSPACE;
-  }
-  fp8blk_status st = make_launch(stream, L);
+  st = make_launch(stream, L);
   if (st != FP8BLK_OK) return st;
   if (K == 0) {  // empty sum: y = 0
     *done = true;

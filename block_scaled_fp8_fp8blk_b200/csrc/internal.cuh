@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "fp8blk.h"
+
 namespace fp8blk {
 
 struct Launch {
@@ -48,5 +50,15 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
 
 // Sets the kernel's dynamic shared-memory limit once per device.
 cudaError_t ensure_smem_limit(const void* kernel, size_t bytes);
+
+// The launch context of the current device (checks compute capability 10.x).
+fp8blk_status current_launch(fp8blk_stream stream, Launch* L);
+
+// Argument checks of a linear call (no CUDA call): FP8BLK_OK, INVALID_ARG,
+// ALIGNMENT or WORKSPACE; ws_need is fp8blk_workspace_size of the call.
+fp8blk_status validate_linear(const void* x, int64_t ldx, const uint8_t* q, int64_t ldq,
+                              const float* scale_inv, const void* y, int64_t ldy, int64_t M,
+                              int64_t N, int64_t K, const void* ws, size_t ws_bytes,
+                              size_t ws_need);
 
 }  // namespace fp8blk

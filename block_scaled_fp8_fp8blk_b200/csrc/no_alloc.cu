@@ -27,9 +27,6 @@
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FP8BLK_NOALLOC_SCRATCH_BYTES];
 
 namespace fp8blk {
-
-fp8blk_status current_launch(fp8blk_stream stream, Launch* L);
-
 namespace {
 
 constexpr int kMaxDevices = 64;

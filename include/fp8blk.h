@@ -201,6 +201,65 @@ FP8BLK_EXPORT fp8blk_status fp8blk_linear_w8a8_quantized(const uint8_t* qx, int6
                                                          int64_t ldy, int64_t M, int64_t N,
                                                          int64_t K, fp8blk_stream stream);
 
+/* ---------------------------------------------------------------------------
+ * Layerwise FP8 weight streaming (FastVideo PR #1829, "Purpose": the FP8
+ * checkpoint is what keeps the encoder resident, and what an offloaded
+ * encoder moves instead of BF16 weights; the page reports both the memory
+ * and the offload time of the two forms). Runs a sequence of linears whose
+ * codes and scales live in HOST memory through a ring of `nslots` device
+ * weight slots: job i's weights are copied into slot i % nslots on `copy`
+ * while earlier jobs run on `compute`; job i's linear runs on `compute` once
+ * its copy has landed, and a slot is refilled only after the linear that
+ * read it has finished. Each job computes exactly what fp8blk_linear_w8a16
+ * (mode 0) or fp8blk_linear_w8a8 (mode 1) computes from the same weights on
+ * the device.
+ *   jobs[i].q_host     : uint8 [N][ldq] in HOST memory (pinned, or the
+ *                        copies are not asynchronous), ldq >= K, ldq % 16 == 0
+ *   jobs[i].scale_host : float [ceil(N/128)][ceil(K/128)] in HOST memory
+ *   jobs[i].x, ldx, y, ldy, M, N, K : DEVICE activations and output, as for
+ *                        the linear calls (x read, y written on `compute`)
+ *   slots      : DEVICE, nslots consecutive slots of slot_bytes each;
+ *                256-byte aligned, slot_bytes % 256 == 0 and
+ *                slot_bytes >= fp8blk_stream_slot_bytes(N, K, ldq) of every
+ *                job (codes at the start of a slot, scales after them)
+ *   workspace  : DEVICE, as for the linear calls, at least the largest
+ *                fp8blk_workspace_size(mode, M, N, K) over the jobs
+ *   compute, copy : streams (the same stream twice is valid: no overlap)
+ *   events     : 2 * nslots cudaEvent_t created by the caller (timing
+ *                disabled is best); the library only records and waits on them
+ * The copies of a call start after the work already enqueued on `compute`,
+ * so consecutive calls may share slots and events.
+ * Everything is enqueued asynchronously: on return nothing need have run.
+ * Every job is checked before anything is enqueued; a CUDA error while
+ * enqueuing returns FP8BLK_ERR_CUDA with the jobs before it enqueued.
+ * Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED_DEVICE, CUDA.
+ * ------------------------------------------------------------------------- */
+typedef struct fp8blk_linear_job {
+  int32_t mode;              /* 0 = W8A16, 1 = W8A8 */
+  const uint8_t* q_host;     /* host codes [N][ldq] */
+  const float* scale_host;   /* host scales [ceil(N/128)][ceil(K/128)] */
+  int64_t ldq;
+  const void* x;             /* device BF16 activations [M][ldx] */
+  int64_t ldx;
+  void* y;                   /* device BF16 output [M][ldy] */
+  int64_t ldy;
+  int64_t M, N, K;
+} fp8blk_linear_job;
+
+/* A cudaEvent_t, passed as an opaque pointer. */
+typedef void* fp8blk_event;
+
+/* Bytes of one weight slot for an N x K linear with code pitch ldq: the
+ * codes rounded up to 256 bytes, then the scales, rounded up to 256. Pure
+ * host function; 0 for negative sizes or ldq < K. */
+FP8BLK_EXPORT size_t fp8blk_stream_slot_bytes(int64_t N, int64_t K, int64_t ldq);
+
+FP8BLK_EXPORT fp8blk_status fp8blk_streamed_linears(const fp8blk_linear_job* jobs, int64_t njobs,
+                                                    void* slots, size_t slot_bytes, int32_t nslots,
+                                                    void* workspace, size_t workspace_bytes,
+                                                    fp8blk_stream compute, fp8blk_stream copy,
+                                                    fp8blk_event* events);
+
 /* Workspace bytes for a linear: mode 0 = W8A16, 1 = W8A8. Pure host function;
  * returns 0 for an invalid mode or negative sizes. */
 FP8BLK_EXPORT size_t fp8blk_workspace_size(int mode, int64_t M, int64_t N, int64_t K);

@@ -160,3 +160,48 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(fb, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         fb.lib()
+
+
+def test_stream_slot_bytes(lib):
+    # codes 1000 x 1008 = 1008000 -> 1008128 (256-aligned), + 8 x 8 scales x 4 B
+    assert lib.fp8blk_stream_slot_bytes(1000, 1000, 1008) == 1008128 + 256
+    assert lib.fp8blk_stream_slot_bytes(25600, 5120, 5120) == 25600 * 5120 + 200 * 40 * 4
+    assert lib.fp8blk_stream_slot_bytes(0, 0, 0) == 0
+    assert lib.fp8blk_stream_slot_bytes(16, 64, 32) == 0      # ldq < K
+    assert lib.fp8blk_stream_slot_bytes(-1, 64, 64) == 0
+
+
+def test_streamed_linears_validation(lib):
+    """Every job is checked before any CUDA call, so these run without a GPU."""
+    M, N, K = 64, 384, 256
+    slot = lib.fp8blk_stream_slot_bytes(N, K, K)
+    slot = -(-slot // 256) * 256
+    ws = lib.fp8blk_workspace_size(1, M, N, K)
+    events = (ctypes.c_void_p * 4)(P, P + 16, P + 32, P + 48)
+
+    def job(**kw):
+        d = dict(mode=1, q_host=P, scale_host=P, ldq=K, x=P, ldx=K, y=P, ldy=N, M=M, N=N, K=K)
+        d.update(kw)
+        return fb.LinearJob(**d)
+
+    def call(jobs, njobs=None, slots=P, slot_bytes=slot, nslots=2, wsp=P, wsb=ws, ev=events):
+        arr = (fb.LinearJob * max(1, len(jobs)))(*jobs)
+        return lib.fp8blk_streamed_linears(arr, len(jobs) if njobs is None else njobs, slots,
+                                           slot_bytes, nslots, wsp, wsb, None, None, ev)
+
+    assert call([], njobs=0) == 0
+    assert call([job()], njobs=-1) == 1
+    assert call([job()], nslots=0) == 1
+    assert call([job()], slots=None) == 1
+    assert call([job()], ev=None) == 1
+    assert call([job()], slot_bytes=slot + 16) == 2               # slot size % 256
+    assert call([job()], slots=P + 16) == 2                       # slots 256-byte aligned
+    assert call([job()], ev=(ctypes.c_void_p * 4)(P, None, P, P)) == 1
+    assert call([job(mode=2)]) == 1
+    assert call([job(), job(N=N * 4, ldy=N * 4)]) == 1           # second job's weights exceed a slot
+    assert call([job(ldq=K - 16)]) == 1
+    assert call([job(q_host=None)]) == 1
+    assert call([job(x=PM)]) == 2
+    assert call([job(ldx=K + 4)]) == 2
+    assert call([job()], wsp=None) == 4                           # W8A8 needs its workspace
+    assert call([job()], wsb=ws - 1) == 4

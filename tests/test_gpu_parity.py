@@ -311,3 +311,46 @@ def test_linear_w8a8_quantized_matches_linear_w8a8(wl):
     qx, sx = fb.quantize_act(x_d)
     got = bf16_bits(fb.linear_w8a8_quantized(qx, sx, q_d, s_d))
     assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------------- weight streaming
+STREAM_JOBS = [(0, 64, 1024, 1536), (1, 300, 640, 512), (0, 1, 5120, 2048), (1, 77, 1000, 1000),
+               (0, 200, 384, 640), (0, 16, 256, 384), (1, 8, 2048, 1024)]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("nslots", [1, 2, 3])
+def test_streamed_linears_match_resident(nslots):
+    """Weights streamed from pinned host memory through nslots device slots
+    give exactly what the same linears give on resident weights."""
+    g = torch.Generator(device="cpu").manual_seed(21)
+    jobs, ref, outs, slot = [], [], [], 0
+    ws_need = 0
+    for mode, M, K, N in STREAM_JOBS:
+        w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
+        ldx = -(-K // 8) * 8
+        x = torch.randn(M, ldx, generator=g).to(torch.bfloat16).to(DEV)[:, :K]
+        q, s = fb.quantize_weight(w)
+        ldq = q.stride(0)
+        qh = torch.empty((N, ldq), dtype=torch.uint8, pin_memory=True)
+        qh[:, :K] = q.cpu()
+        sh = s.cpu().pin_memory()
+        f = fb.linear_w8a16 if mode == 0 else fb.linear_w8a8
+        ref.append(f(x, q, s))
+        y = torch.full_like(ref[-1], 7.0)
+        outs.append(y)
+        jobs.append((mode, qh[:, :K], sh, x, y))
+        slot = max(slot, fb.stream_slot_bytes(N, K, ldq))
+        ws_need = max(ws_need, fb.workspace_size(mode, M, N, K))
+    slot = -(-slot // 256) * 256
+    slots = torch.empty(nslots * slot, dtype=torch.uint8, device=DEV)
+    ws = torch.empty(max(1, ws_need), dtype=torch.uint8, device=DEV)
+    compute, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    events = [torch.cuda.Event() for _ in range(2 * nslots)]
+    compute.wait_stream(torch.cuda.current_stream())
+    fb.streamed_linears(jobs, slots, slot, nslots, ws, compute, copy, events)
+    torch.cuda.current_stream().wait_stream(compute)
+    torch.cuda.synchronize()
+    for (mode, M, K, N), r, y in zip(STREAM_JOBS, ref, outs):
+        assert torch.equal(y.view(torch.int16), r.view(torch.int16)), (mode, M, K, N)
+    assert fb.read_device_error() == 0
