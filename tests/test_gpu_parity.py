@@ -354,3 +354,39 @@ def test_streamed_linears_match_resident(nslots):
     for (mode, M, K, N), r, y in zip(STREAM_JOBS, ref, outs):
         assert torch.equal(y.view(torch.int16), r.view(torch.int16)), (mode, M, K, N)
     assert fb.read_device_error() == 0
+
+
+# ----------------------------------------------------------- checkpoints
+@pytest.mark.gpu
+def test_checkpoint_conversion_matches_oracle(tmp_path):
+    """BF16 checkpoint -> block-FP8 checkpoint on the GPU: every converted
+    weight's codes and scales equal the oracle's, other tensors pass through,
+    and a linear on the loaded weights equals one on the in-memory weights."""
+    from block_scaled_fp8_fp8blk_b200 import checkpoint as ck
+    g = torch.Generator(device="cpu").manual_seed(31)
+    src = {
+        "model.layers.0.self_attn.q_proj.weight": (torch.randn(384, 256, generator=g) * 0.02).to(torch.bfloat16),
+        "model.layers.0.mlp.down_proj.weight": (torch.randn(300, 1000, generator=g) * 0.02).to(torch.bfloat16),
+        "model.layers.0.input_layernorm.weight": torch.randn(256, generator=g).to(torch.bfloat16),
+        "model.embed_tokens.weight": torch.randn(40, 256, generator=g).to(torch.bfloat16),
+    }
+    src_dir, dst_dir = str(tmp_path / "bf16"), str(tmp_path / "fp8")
+    ck.save_checkpoint(src_dir, src, config={"model_type": "synthetic"})
+    ck.convert_checkpoint(src_dir, dst_dir, max_shard_bytes=300_000)
+    got, cfg = ck.load_checkpoint(dst_dir)
+    assert cfg["quantization_config"]["weight_block_size"] == [128, 128]
+    for name, w in src.items():
+        if not ck.default_is_linear(name, w):
+            assert torch.equal(got[name].view(torch.int16), w.view(torch.int16))
+            assert name + "_scale_inv" not in got
+            continue
+        q_ref, s_ref = oracle.quantize_weight(w.view(torch.int16).numpy().view(np.uint16))
+        assert np.array_equal(got[name].view(torch.uint8).numpy(), q_ref)
+        assert np.array_equal(got[name + "_scale_inv"].numpy().view(np.uint32), s_ref.view(np.uint32))
+    name = "model.layers.0.mlp.down_proj.weight"
+    q, s = ck.linear_weights(got, name)
+    x = torch.randn(64, 1008, generator=g).to(torch.bfloat16).to(DEV)[:, :1000]
+    q_direct, s_direct = fb.quantize_weight(
+        torch.nn.functional.pad(src[name], (0, 8)).to(DEV)[:, :1000])
+    for f in (fb.linear_w8a16, fb.linear_w8a8):
+        assert torch.equal(f(x, q, s).view(torch.int16), f(x, q_direct, s_direct).view(torch.int16))
