@@ -17,7 +17,7 @@ import os
 __all__ = [
     "Fp8BlkError", "lib", "quantize_weight", "dequantize", "quantize_act", "linear_w8a16",
     "linear_w8a8", "linear_w8a8_quantized", "workspace_size", "encode_e4m3", "read_device_error",
-    "version", "LinearJob", "stream_slot_bytes", "streamed_linears",
+    "version", "LinearJob", "stream_slot_bytes", "streamed_linears", "selftest_wait_timeout",
     "LIB_PATH", "EXPORTS",
 ]
 
@@ -56,6 +56,7 @@ EXPORTS = {
                                       _p, _sz, _p, _p, ctypes.POINTER(_p)]),
     "fp8blk_encode_e4m3": (_st, [_p, _i64, _p, _p]),
     "fp8blk_read_device_error": (_st, [ctypes.POINTER(ctypes.c_uint32)]),
+    "fp8blk_selftest_wait_timeout": (_st, [_i64, _p]),
     "fp8blk_status_string": (ctypes.c_char_p, [_int]),
     "fp8blk_version": (_int, []),
 }
@@ -243,6 +244,12 @@ def encode_e4m3(v):
     _check(lib().fp8blk_encode_e4m3(v.data_ptr(), v.numel(), out.data_ptr(), _stream()),
            "fp8blk_encode_e4m3")
     return out
+
+
+def selftest_wait_timeout(limit_cycles: int = 2_000_000) -> None:
+    """Launches the failure-detection self-test (a bounded wait that runs out)."""
+    _check(lib().fp8blk_selftest_wait_timeout(limit_cycles, _stream()),
+           "fp8blk_selftest_wait_timeout")
 
 
 def read_device_error() -> int:

@@ -11,11 +11,25 @@
 
 #include "fp8blk.h"
 #include "internal.cuh"
+#include "ptx.cuh"
 
 namespace fp8blk {
 
 // Bit flags set by kernels whose bounded waits ran out (see ptx.cuh).
 __device__ unsigned g_device_error = 0;
+
+// The failure-detection path on its own: one warp waits, with the kernels'
+// bounded wait, on an mbarrier phase that nothing completes; the wait gives
+// up after limit_cycles, sets kErrWaitSelfTest and the kernel returns.
+__global__ void selftest_wait_kernel(unsigned* err, long long limit_cycles) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);  // one arrival expected; none comes
+    mbar_init_fence();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_wait_for(&bar, 0u, err, kErrWaitSelfTest, limit_cycles);
+}
 
 namespace {
 
@@ -310,6 +324,15 @@ fp8blk_status fp8blk_encode_e4m3(const float* v, int64_t n, uint8_t* codes, fp8b
   fp8blk_status st = make_launch(stream, &L);
   if (st != FP8BLK_OK) return st;
   return cuda_status(launch_encode_e4m3(L, v, n, codes));
+}
+
+fp8blk_status fp8blk_selftest_wait_timeout(int64_t limit_cycles, fp8blk_stream stream) {
+  if (limit_cycles < 1000 || limit_cycles > kWaitLimitCycles) return FP8BLK_ERR_INVALID_ARG;
+  Launch L;
+  fp8blk_status st = make_launch(stream, &L);
+  if (st != FP8BLK_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, L.stream>>>(L.err, limit_cycles);
+  return cuda_status(cudaGetLastError());
 }
 
 fp8blk_status fp8blk_read_device_error(uint32_t* word) {

@@ -18,6 +18,7 @@ enum DeviceErrorBits : unsigned {
   kErrWaitMma = 2u,
   kErrWaitEpilogue = 4u,
   kErrWaitExpand = 8u,
+  kErrWaitSelfTest = 16u,
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -58,9 +59,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete, at most
-// kWaitLimitCycles; on time-out OR `flag` into *err and return false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
-                                          unsigned flag) {
+// limit_cycles; on time-out OR `flag` into *err and return false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned* err,
+                                              unsigned flag, long long limit_cycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
@@ -71,11 +72,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
       __nanosleep(FP8BLK_WAIT_BACKOFF_NS);
 #endif
     }
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit_cycles) {
       atomicOr(err, flag);
       return false;
     }
   }
+}
+
+// The kernels' wait: at most kWaitLimitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
+                                          unsigned flag) {
+  return mbar_wait_for(bar, parity, err, flag, kWaitLimitCycles);
 }
 
 // Bounded wait for a thread that is normally far ahead of the barrier it

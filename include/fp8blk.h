@@ -273,8 +273,18 @@ FP8BLK_EXPORT size_t fp8blk_workspace_size(int mode, int64_t M, int64_t N, int64
  * ------------------------------------------------------------------------- */
 FP8BLK_EXPORT fp8blk_status fp8blk_encode_e4m3(const float* v, int64_t n, uint8_t* codes, fp8blk_stream stream);
 
+/* Self-test of the failure-detection path: launches one warp that waits, with
+ * the kernels' own bounded wait, on an mbarrier phase that nothing completes.
+ * After limit_cycles SM cycles (1000 <= limit_cycles <= 4e9; a few million is
+ * about a millisecond) the wait gives up, sets flag 16 in the error word and
+ * the kernel returns, leaving the context usable: fp8blk_read_device_error
+ * then reports FP8BLK_ERR_TIMEOUT with word 16. No fault, trap or hang.
+ * Errors: INVALID_ARG, UNSUPPORTED_DEVICE, CUDA. */
+FP8BLK_EXPORT fp8blk_status fp8blk_selftest_wait_timeout(int64_t limit_cycles, fp8blk_stream stream);
+
 /* Reads and clears the current device's error word (bit flags set by a kernel
- * whose bounded wait ran out: 1 load, 2 MMA, 4 epilogue, 8 weight expansion).
+ * whose bounded wait ran out: 1 load, 2 MMA, 4 epilogue, 8 weight expansion,
+ * 16 the self-test above).
  * Synchronizes the device. *word receives the flags; returns FP8BLK_ERR_TIMEOUT
  * when any flag was set, FP8BLK_OK when none, FP8BLK_ERR_CUDA on a CUDA error. */
 FP8BLK_EXPORT fp8blk_status fp8blk_read_device_error(uint32_t* word);

@@ -205,3 +205,8 @@ def test_streamed_linears_validation(lib):
     assert call([job(ldx=K + 4)]) == 2
     assert call([job()], wsp=None) == 4                           # W8A8 needs its workspace
     assert call([job()], wsb=ws - 1) == 4
+
+
+def test_selftest_wait_timeout_validation(lib):
+    assert lib.fp8blk_selftest_wait_timeout(999, None) == 1
+    assert lib.fp8blk_selftest_wait_timeout(4_000_000_001, None) == 1

@@ -390,3 +390,18 @@ def test_checkpoint_conversion_matches_oracle(tmp_path):
         torch.nn.functional.pad(src[name], (0, 8)).to(DEV)[:, :1000])
     for f in (fb.linear_w8a16, fb.linear_w8a8):
         assert torch.equal(f(x, q, s).view(torch.int16), f(x, q_direct, s_direct).view(torch.int16))
+
+
+# ------------------------------------------------------ failure detection
+@pytest.mark.gpu
+def test_bounded_wait_times_out_and_context_stays_usable():
+    """A wait that nothing completes gives up after its limit, reports through
+    the device error word, and the context keeps working afterwards."""
+    assert fb.read_device_error() == 0
+    fb.selftest_wait_timeout(2_000_000)          # about a millisecond
+    torch.cuda.synchronize()
+    assert fb.read_device_error() == 16
+    assert fb.read_device_error() == 0           # read-and-clear
+    wl = W.RAGGED
+    run_linear(wl, "w8a16")                       # still correct after the time-out
+    assert fb.read_device_error() == 0
