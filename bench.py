@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--stack", type=int, default=0,
                     help="instead of the step: stream the FP8 weights of this many 32B-shaped "
                          "layers from pinned host memory (one GPU)")
+    ap.add_argument("--decode", type=int, default=0,
+                    help="instead of the step: one 32B-shaped layer's four linears at this many "
+                         "tokens, as separate calls, as one sequence, and as a CUDA graph of it")
     ap.add_argument("--stack-mode", type=int, default=0, choices=[0, 1], help="0 W8A16, 1 W8A8")
     ap.add_argument("--stack-m", type=int, default=512)
     ap.add_argument("--stack-slots", type=int, default=2)
@@ -314,6 +317,87 @@ def stack_arm(args):
     print(json.dumps(line), flush=True)
 
 
+def decode_arm(args):
+    """One decoder layer of the 32B class at a small token count: the weight
+    stream (487.7 MB of FP8 codes per layer) is the whole cost. Timed as four
+    separate linear calls, as one fp8blk_linear_sequence (each GEMM streams
+    its weights while the kernel before it ends), and as a CUDA graph of that
+    sequence; L2 flushed (memset + read) before each timed layer."""
+    import torch
+    import block_scaled_fp8_fp8blk_b200 as fb
+    M, mode = args.decode, args.stack_mode
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(7)
+    jobs, wbytes, ws_need = [], 0, 0
+    for name, K, N in STACK_LAYER:
+        ldq = -(-K // 16) * 16
+        q = (torch.randint(0, 0x7F, (N, ldq), device=dev, generator=g, dtype=torch.uint8)
+             | (torch.randint(0, 2, (N, ldq), device=dev, generator=g, dtype=torch.uint8) << 7))[:, :K]
+        s = torch.rand(-(-N // 128), -(-K // 128), device=dev, generator=g) * 1e-3 + 1e-4
+        x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        jobs.append((mode, x, q, s, y))
+        wbytes += N * K + 4 * s.numel()
+        ws_need = max(ws_need, fb.workspace_size(mode, M, N, K))
+    ws = torch.empty(max(1, ws_need), dtype=torch.uint8, device=dev)
+    f = fb.linear_w8a16 if mode == 0 else fb.linear_w8a8
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def separate():
+        for m_, x, q, s, y in jobs:
+            f(x, q, s, out=y, workspace=ws)
+
+    def sequence():
+        fb.linear_sequence(jobs, workspace=ws)
+
+    for run in (separate, sequence):
+        run()
+    torch.cuda.synchronize()
+    cs = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cs):
+        sequence()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=cs):
+            sequence()
+    torch.cuda.synchronize()
+    reps = max(5, min(args.steps, 50))
+
+    def timed(run):
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            flush_rd.sum()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(); run(); b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return 1e3 * statistics.median(a.elapsed_time(b) for a, b in ts)
+
+    res = {"separate_calls": timed(separate), "sequence": timed(sequence),
+           "sequence_cuda_graph": timed(graph.replay)}
+    assert fb.read_device_error() == 0
+    peaks, peak_kind = load_peaks()
+    line = {
+        "metric": "decode layer: weight-stream GB/s (4 linears of a 32B-class layer, FP8 weights)",
+        "value": wbytes / (res["sequence"] * 1e-6) / 1e9, "unit": "GB/s", "higher_is_better": True,
+        "n_gpus": 1, "steps": reps, "data": "synthetic (random finite E4M3 codes and scales)",
+        "dtype": "e4m3 weights, bf16 activations" if mode == 0 else "e4m3 weights and activations",
+        "config": {"workload": f"decode_layer32b_m{M}", "M": M,
+                   "shapes_KN": [[k, n] for _, k, n in STACK_LAYER],
+                   "mode": "w8a16" if mode == 0 else "w8a8",
+                   "l2": "flushed (memset + read) before each timed layer"},
+        "weight_bytes_per_layer": wbytes,
+        "us_per_layer": res,
+        "weight_stream_gbs": {k: wbytes / (v * 1e-6) / 1e9 for k, v in res.items()},
+        "hbm_frac": {k: wbytes / (v * 1e-6) / 1e9 / peaks["hbm_gbs"] for k, v in res.items()},
+        "peak_gbs": peaks["hbm_gbs"], "peak_kind": peak_kind,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     from block_scaled_fp8_fp8blk_b200 import workloads
@@ -321,6 +405,10 @@ def main():
     if args.stack > 0:
         if int(os.environ.get("RANK", "0")) == 0:
             stack_arm(args)
+        return
+    if args.decode > 0:
+        if int(os.environ.get("RANK", "0")) == 0:
+            decode_arm(args)
         return
     if args.impl == "reference":
         return reference_arm(args, wl)

@@ -18,6 +18,7 @@ __all__ = [
     "Fp8BlkError", "lib", "quantize_weight", "dequantize", "quantize_act", "linear_w8a16",
     "linear_w8a8", "linear_w8a8_quantized", "workspace_size", "encode_e4m3", "read_device_error",
     "version", "LinearJob", "stream_slot_bytes", "streamed_linears", "selftest_wait_timeout",
+    "LinearArgs", "linear_sequence",
     "LIB_PATH", "EXPORTS",
 ]
 
@@ -41,6 +42,12 @@ class LinearJob(ctypes.Structure):
                 ("M", _i64), ("N", _i64), ("K", _i64)]
 
 
+class LinearArgs(ctypes.Structure):
+    """fp8blk_linear_args: one linear of a sequence (device weights)."""
+    _fields_ = [("mode", ctypes.c_int32), ("x", _p), ("ldx", _i64), ("q", _p), ("ldq", _i64),
+                ("scale_inv", _p), ("y", _p), ("ldy", _i64), ("M", _i64), ("N", _i64), ("K", _i64)]
+
+
 # name -> (restype, argtypes), mirroring include/fp8blk.h
 EXPORTS = {
     "fp8blk_quantize_weight": (_st, [_p, _i64, _i64, _i64, _p, _i64, _p, _p]),
@@ -52,6 +59,7 @@ EXPORTS = {
     "fp8blk_linear_w8a8_quantized": (_st, [_p, _i64, _p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p]),
     "fp8blk_workspace_size": (_sz, [_int, _i64, _i64, _i64]),
     "fp8blk_stream_slot_bytes": (_sz, [_i64, _i64, _i64]),
+    "fp8blk_linear_sequence": (_st, [ctypes.POINTER(LinearArgs), _i64, _p, _sz, _p]),
     "fp8blk_streamed_linears": (_st, [ctypes.POINTER(LinearJob), _i64, _p, _sz, ctypes.c_int32,
                                       _p, _sz, _p, _p, ctypes.POINTER(_p)]),
     "fp8blk_encode_e4m3": (_st, [_p, _i64, _p, _p]),
@@ -202,6 +210,31 @@ def linear_w8a8_quantized(qx, sx, q, scale_inv, M=None, out=None):
                                               out.data_ptr(), _ld(out), M, N, K, _stream()),
            "fp8blk_linear_w8a8_quantized")
     return out
+
+
+def linear_sequence(jobs, workspace=None):
+    """Runs linears back to back with their weight streams overlapping the
+    kernels before them (fp8blk_linear_sequence). jobs: list of
+    (mode, x, q, scale_inv, y) with mode 0 = W8A16, 1 = W8A8, all CUDA
+    tensors as for linear_w8a16 / linear_w8a8. The workspace (allocated here
+    if None) must cover the largest workspace_size over the jobs."""
+    import torch
+    arr = (LinearArgs * max(1, len(jobs)))()
+    need = 0
+    for i, (mode, x, q, s, y) in enumerate(jobs):
+        M, K = x.shape
+        N = q.shape[0]
+        if q.shape[1] != K or y.shape != (M, N):
+            raise ValueError("job shapes disagree")
+        arr[i] = LinearArgs(mode, x.data_ptr(), _ld(x), q.data_ptr(), _ld(q), s.data_ptr(),
+                            y.data_ptr(), _ld(y), M, N, K)
+        need = max(need, workspace_size(mode, M, N, K))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=jobs[0][1].device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().fp8blk_linear_sequence(arr, len(jobs), ws_ptr, ws_len, _stream()),
+           "fp8blk_linear_sequence")
 
 
 def stream_slot_bytes(N: int, K: int, ldq: int) -> int:

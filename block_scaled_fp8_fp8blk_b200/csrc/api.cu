@@ -279,6 +279,56 @@ fp8blk_status fp8blk_linear_w8a8(const void* x, int64_t ldx, const uint8_t* q, i
                                       static_cast<uint16_t*>(y), ldy, M, N, K, true));
 }
 
+fp8blk_status fp8blk_linear_sequence(const fp8blk_linear_args* jobs, int64_t njobs,
+                                     void* workspace, size_t workspace_bytes,
+                                     fp8blk_stream stream) {
+  if (njobs < 0) return FP8BLK_ERR_INVALID_ARG;
+  if (njobs == 0) return FP8BLK_OK;
+  if (!jobs) return FP8BLK_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < njobs; ++i) {
+    const fp8blk_linear_args& j = jobs[i];
+    if (j.mode != 0 && j.mode != 1) return FP8BLK_ERR_INVALID_ARG;
+    const fp8blk_status st = validate_linear(j.x, j.ldx, j.q, j.ldq, j.scale_inv, j.y, j.ldy, j.M,
+                                             j.N, j.K, workspace, workspace_bytes,
+                                             fp8blk_workspace_size(j.mode, j.M, j.N, j.K));
+    if (st != FP8BLK_OK) return st;
+  }
+  Launch L;
+  fp8blk_status st = make_launch(stream, &L);
+  if (st != FP8BLK_OK) return st;
+  // The first kernel waits for everything before the call; after it, each
+  // GEMM may read its (read-only) weights before the kernel before it ends.
+  bool first = true;
+  for (int64_t i = 0; i < njobs; ++i) {
+    const fp8blk_linear_args& j = jobs[i];
+    if (j.M == 0 || j.N == 0) continue;
+    if (j.K == 0) {
+      if (cudaMemset2DAsync(j.y, static_cast<size_t>(j.ldy) * 2, 0, static_cast<size_t>(j.N) * 2,
+                            static_cast<size_t>(j.M), L.stream) != cudaSuccess)
+        return FP8BLK_ERR_CUDA;
+      continue;
+    }
+    cudaError_t e;
+    if (j.mode == 0) {
+      e = launch_w8a16_gemm(L, static_cast<const uint16_t*>(j.x), j.ldx, j.q, j.ldq, j.scale_inv,
+                            static_cast<uint16_t*>(j.y), j.ldy, j.M, j.N, j.K, workspace,
+                            workspace_bytes, !first);
+    } else {
+      uint8_t* qx = static_cast<uint8_t*>(workspace);
+      float* sx = reinterpret_cast<float*>(qx + w8a8_sx_offset(j.M, j.K));
+      const int64_t ldqx = w8a8_ldqx(j.K), ldsx = w8a8_ldsx(j.M);
+      e = launch_quantize_act(L, static_cast<const uint16_t*>(j.x), j.M, j.K, j.ldx, qx, ldqx, sx,
+                              ldsx, !first);
+      if (e == cudaSuccess)
+        e = launch_w8a8_gemm(L, qx, ldqx, sx, ldsx, j.q, j.ldq, j.scale_inv,
+                             static_cast<uint16_t*>(j.y), j.ldy, j.M, j.N, j.K, true);
+    }
+    if (e != cudaSuccess) return FP8BLK_ERR_CUDA;
+    first = false;
+  }
+  return FP8BLK_OK;
+}
+
 fp8blk_status fp8blk_linear_w8a8_quantized(const uint8_t* qx, int64_t ldqx, const float* sx,
                                            int64_t ldsx, const uint8_t* q, int64_t ldq,
                                            const float* scale_inv, void* y, int64_t ldy, int64_t M,

@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(512, 1)
     w8a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_x,
                       const float* __restrict__ sw, __nv_bfloat16* __restrict__ y, int64_t ldy,
                       int M, int N, int KB, int mtiles, int ntiles_total, int streamk,
-                      float* __restrict__ part, unsigned* __restrict__ err) {
+                      int early_weights, float* __restrict__ part, unsigned* __restrict__ err) {
   using C = W8A16Cfg<BT, NSUB>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
@@ -258,8 +258,13 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  // The stream-K fix-up kernel may be scheduled now; it waits for this grid.
-  if (streamk) pdl_launch_dependents();
+  // The kernel after this one in the stream (the stream-K fix-up, or the
+  // next linear) may be scheduled now: whatever it reads of this kernel's
+  // output it reads after griddepcontrol.wait. This kernel in turn reads the
+  // activations, and writes y and the workspace, only after its own wait for
+  // the kernel before it; the weights too, unless the caller has promised
+  // that the kernel before does not write them (early_weights).
+  pdl_launch_dependents();
 
   // Each warpgroup sets its register budget at the top of its role:
   // 128 x (56 + 80 + 184 + 184) = 64512 of the 65536 the block holds.
@@ -269,6 +274,7 @@ __global__ void __launch_bounds__(512, 1)
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------ weight-code producer
       tma_prefetch_map(&tm_q);
+      if (!early_weights) pdl_wait();
       int j = 0;  // slab counter (across tiles)
       bool ok = true;
       Schedule sc(streamk != 0, KB, ntiles_total);
@@ -291,6 +297,7 @@ __global__ void __launch_bounds__(512, 1)
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------- activation producer
       tma_prefetch_map(&tm_x);
+      pdl_wait();
       int i = 0;  // item counter (across tiles)
       bool ok = true;
       Schedule sc(streamk != 0, KB, ntiles_total);
@@ -362,6 +369,7 @@ __global__ void __launch_bounds__(512, 1)
     setmaxnreg_inc<184>();
     if constexpr (NSUB == 2) {
       // ------------------------------------ promotion/epilogue (two sub-tiles)
+      pdl_wait();  // y may still be read by the kernel before
       // All eight warps promote every item: warp 8 + 4h + q owns TMEM lane
       // quadrant q and token columns [64h, 64h + 64) of each item's partial,
       // so a partial is read by eight warps at once (two 32-column loads
@@ -438,6 +446,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     } else if (((warp - 8) >> 2) < NSUB) {
       // ------------------------------------------------ promotion/epilogue
+      pdl_wait();  // y and the workspace may still be in use by the kernel before
       const int t = (warp - 8) >> 2;  // token sub-tile
       const int quad = warp & 3;
       const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::TMEM_P;
@@ -593,6 +602,7 @@ __global__ void __launch_bounds__(256) w8a16_streamk_fixup(const __grid_constant
                                                            const float* __restrict__ part,
                                                            uint16_t* __restrict__ y, int64_t ldy,
                                                            int M, int N) {
+  pdl_launch_dependents();  // the next linear may be scheduled; it waits for this grid
   pdl_wait();
   const int i = static_cast<int>(blockIdx.x);
   const int r = threadIdx.x & 127;
@@ -626,7 +636,7 @@ __global__ void __launch_bounds__(256) w8a16_streamk_fixup(const __grid_constant
 template <int BT, int NSUB>
 cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                       int64_t ldq, const float* sw, uint16_t* y, int64_t ldy, int64_t M,
-                      int64_t N, int64_t K, void* ws, size_t ws_bytes) {
+                      int64_t N, int64_t K, void* ws, size_t ws_bytes, bool early_weights) {
   using C = W8A16Cfg<BT, NSUB>;
   CUtensorMap tq, tx;
   if (!make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, N, ldq, 128, 128))
@@ -660,12 +670,26 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
   if (grid > cap) grid = cap;
   if (streamk && (!ws || ws_bytes < static_cast<size_t>(grid) * 2 * BT * 128 * sizeof(float)))
     return cudaErrorInvalidValue;
-  kern<<<static_cast<int>(grid), C::THREADS, C::SMEM, L.stream>>>(
-      tq, tx, sw, reinterpret_cast<__nv_bfloat16*>(y), ldy, static_cast<int>(M),
-      static_cast<int>(N), static_cast<int>(KB), static_cast<int>(mtiles),
-      static_cast<int>(tiles), streamk ? 1 : 0, static_cast<float*>(ws), L.err);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || !streamk || grid < 2) return e;
+  // A programmatic dependent of the kernel before it in the stream (its set-up
+  // overlaps that kernel's tail; see the kernel for what waits).
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, tq, tx, sw, reinterpret_cast<__nv_bfloat16*>(y), ldy,
+                           static_cast<int>(M), static_cast<int>(N), static_cast<int>(KB),
+                           static_cast<int>(mtiles), static_cast<int>(tiles), streamk ? 1 : 0,
+                           early_weights ? 1 : 0, static_cast<float*>(ws), L.err);
+    if (e != cudaSuccess) return e;
+  }
+  if (!streamk || grid < 2) return cudaSuccess;
   const SplitTiles st = split_tiles(tiles, KB, grid);
   if (st.count == 0) return cudaSuccess;
   const int mt = static_cast<int>(M < BT ? M : BT);
@@ -697,12 +721,12 @@ size_t w8a16_workspace_bytes(int64_t M, int64_t, int64_t) {
 
 cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                               int64_t ldq, const float* sw, uint16_t* y, int64_t ldy, int64_t M,
-                              int64_t N, int64_t K, void* ws, size_t ws_bytes) {
-  if (M <= 16) return launch_bt<16, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
-  if (M <= 32) return launch_bt<32, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
-  if (M <= 64) return launch_bt<64, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
-  if (M <= 128) return launch_bt<128, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
-  return launch_bt<128, 2>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes);
+                              int64_t N, int64_t K, void* ws, size_t ws_bytes, bool early_weights) {
+  if (M <= 16) return launch_bt<16, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  if (M <= 32) return launch_bt<32, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  if (M <= 64) return launch_bt<64, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  if (M <= 128) return launch_bt<128, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  return launch_bt<128, 2>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
 }
 
 }  // namespace fp8blk

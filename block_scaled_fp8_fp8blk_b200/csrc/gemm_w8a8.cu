@@ -119,6 +119,9 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // The next kernel in the stream may be scheduled now; it reads y after its
+  // own griddepcontrol.wait.
+  pdl_launch_dependents();
 
   // Each warpgroup sets its register budget at the top of its role.
   if (warp < 4) {

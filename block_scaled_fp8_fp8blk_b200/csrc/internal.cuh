@@ -24,8 +24,11 @@ cudaError_t launch_quantize_weight(const Launch& L, const uint16_t* w, int64_t N
 cudaError_t launch_dequantize(const Launch& L, const uint8_t* q, int64_t ldq,
                               const float* scale_inv, int64_t N, int64_t K, uint16_t* w,
                               int64_t ldw);
+// pdl: launched as a programmatic dependent of the kernel before it (which
+// may still be running; the kernel reads x only after griddepcontrol.wait).
 cudaError_t launch_quantize_act(const Launch& L, const uint16_t* x, int64_t M, int64_t K,
-                                int64_t ldx, uint8_t* qx, int64_t ldqx, float* sx, int64_t ldsx);
+                                int64_t ldx, uint8_t* qx, int64_t ldqx, float* sx, int64_t ldsx,
+                                bool pdl = false);
 cudaError_t launch_encode_e4m3(const Launch& L, const float* v, int64_t n, uint8_t* codes);
 
 // after_act_quant: launched right after launch_quantize_act on the same
@@ -36,9 +39,13 @@ cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, c
                              bool after_act_quant);
 
 size_t w8a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+// Always a programmatic dependent of the kernel before it; early_weights:
+// that kernel does not write q or scale_inv, so the weight stream may start
+// before it has completed (x, y and the workspace still wait for it).
 cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                               int64_t ldq, const float* scale_inv, uint16_t* y, int64_t ldy,
-                              int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes);
+                              int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
+                              bool early_weights = false);
 
 // 2-D tiled tensor map (128-byte swizzling unless stated) over a row-major
 // matrix [outer][inner] whose rows are row_bytes apart; out-of-bounds reads

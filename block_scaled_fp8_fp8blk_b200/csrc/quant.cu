@@ -293,8 +293,11 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
                                                            float* __restrict__ sx, int64_t ldsx,
                                                            int KB) {
   // The W8A8 GEMM launched after this kernel may be scheduled now: it reads
-  // the codes and scales only after griddepcontrol.wait.
+  // the codes and scales only after griddepcontrol.wait. When this kernel is
+  // itself a programmatic dependent (inside a sequence of linears), x may be
+  // the previous linear's output: wait for that kernel first.
   pdl_launch_dependents();
+  pdl_wait();
   const int j = threadIdx.x & 15;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * 16 + (threadIdx.x >> 4);
   const bool live = g < M * KB;
@@ -365,12 +368,22 @@ cudaError_t launch_dequantize(const Launch& L, const uint8_t* q, int64_t ldq,
 }
 
 cudaError_t launch_quantize_act(const Launch& L, const uint16_t* x, int64_t M, int64_t K,
-                                int64_t ldx, uint8_t* qx, int64_t ldqx, float* sx, int64_t ldsx) {
+                                int64_t ldx, uint8_t* qx, int64_t ldqx, float* sx, int64_t ldsx,
+                                bool pdl) {
   const int64_t ctas = cdiv(M * cdiv(K, 128), 16);
   if (ctas > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  quantize_act_kernel<<<static_cast<unsigned>(ctas), 256, 0, L.stream>>>(
-      x, M, K, ldx, qx, ldqx, sx, ldsx, static_cast<int>(cdiv(K, 128)));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, quantize_act_kernel, x, M, K, ldx, qx, ldqx, sx, ldsx,
+                            static_cast<int>(cdiv(K, 128)));
 }
 
 cudaError_t launch_encode_e4m3(const Launch& L, const float* v, int64_t n, uint8_t* codes) {

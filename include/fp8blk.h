@@ -202,6 +202,40 @@ FP8BLK_EXPORT fp8blk_status fp8blk_linear_w8a8_quantized(const uint8_t* qx, int6
                                                          int64_t K, fp8blk_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * A sequence of linears on device weights, launched back to back so that each
+ * GEMM starts streaming its weights while the kernels before it finish
+ * (programmatic dependent launch). This is the decode-time case: the weight
+ * stream is the whole cost, and the linears of a layer follow one another.
+ * Each job computes exactly what fp8blk_linear_w8a16 (mode 0) or
+ * fp8blk_linear_w8a8 (mode 1) computes from the same arguments, in job order;
+ * a job's x may be an earlier job's y, and a job's y may overwrite an
+ * earlier job's x. The caller promises that no job writes another job's
+ * weights (q, scale_inv): weights are read before the previous job has
+ * finished. The first job waits for all earlier work on `stream`.
+ *   jobs      : njobs job descriptions (host memory), each as for the linear
+ *               calls (device pointers)
+ *   workspace : DEVICE, at least the largest fp8blk_workspace_size(mode, M,
+ *               N, K) over the jobs (the jobs use it one after another)
+ * Every job is checked before anything is launched.
+ * Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED_DEVICE, CUDA.
+ * ------------------------------------------------------------------------- */
+typedef struct fp8blk_linear_args {
+  int32_t mode;              /* 0 = W8A16, 1 = W8A8 */
+  const void* x;             /* BF16 [M][ldx] */
+  int64_t ldx;
+  const uint8_t* q;          /* E4M3 codes [N][ldq] */
+  int64_t ldq;
+  const float* scale_inv;    /* [ceil(N/128)][ceil(K/128)] */
+  void* y;                   /* BF16 [M][ldy] */
+  int64_t ldy;
+  int64_t M, N, K;
+} fp8blk_linear_args;
+
+FP8BLK_EXPORT fp8blk_status fp8blk_linear_sequence(const fp8blk_linear_args* jobs, int64_t njobs,
+                                                   void* workspace, size_t workspace_bytes,
+                                                   fp8blk_stream stream);
+
+/* ---------------------------------------------------------------------------
  * Layerwise FP8 weight streaming (FastVideo PR #1829, "Purpose": the FP8
  * checkpoint is what keeps the encoder resident, and what an offloaded
  * encoder moves instead of BF16 weights; the page reports both the memory

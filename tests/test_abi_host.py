@@ -210,3 +210,27 @@ def test_streamed_linears_validation(lib):
 def test_selftest_wait_timeout_validation(lib):
     assert lib.fp8blk_selftest_wait_timeout(999, None) == 1
     assert lib.fp8blk_selftest_wait_timeout(4_000_000_001, None) == 1
+
+
+def test_linear_sequence_validation(lib):
+    M, N, K = 64, 384, 256
+    ws = lib.fp8blk_workspace_size(1, M, N, K)
+
+    def job(**kw):
+        d = dict(mode=1, x=P, ldx=K, q=P, ldq=K, scale_inv=P, y=P, ldy=N, M=M, N=N, K=K)
+        d.update(kw)
+        return fb.LinearArgs(**d)
+
+    def call(jobs, njobs=None, wsp=P, wsb=ws):
+        arr = (fb.LinearArgs * max(1, len(jobs)))(*jobs)
+        return lib.fp8blk_linear_sequence(arr, len(jobs) if njobs is None else njobs, wsp, wsb, None)
+
+    assert call([], njobs=0) == 0
+    assert call([job()], njobs=-1) == 1
+    assert lib.fp8blk_linear_sequence(None, 1, P, ws, None) == 1
+    assert call([job(mode=3)]) == 1
+    assert call([job(), job(x=PM)]) == 2            # every job checked before any launch
+    assert call([job(), job(ldq=K + 8)]) == 2
+    assert call([job(), job(y=None)]) == 1
+    assert call([job()], wsp=None) == 4
+    assert call([job(mode=0, M=16)], wsp=None) == 4  # W8A16 stream-K needs the workspace too

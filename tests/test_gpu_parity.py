@@ -405,3 +405,39 @@ def test_bounded_wait_times_out_and_context_stays_usable():
     wl = W.RAGGED
     run_linear(wl, "w8a16")                       # still correct after the time-out
     assert fb.read_device_error() == 0
+
+
+# ------------------------------------------------------- linear sequences
+@pytest.mark.gpu
+@pytest.mark.parametrize("M", [1, 64, 300])
+def test_linear_sequence_matches_separate_calls(M):
+    """A chain of linears (each x the previous y, modes mixed) launched as one
+    sequence, weights streamed ahead of the previous kernel's end, gives
+    exactly what separate calls give."""
+    g = torch.Generator(device="cpu").manual_seed(41 + M)
+    dims = [1024, 2048, 640, 1000, 1536]
+    modes = [0, 1, 0, 0, 1, 0][:len(dims) - 1]
+    weights = []
+    for (K, N) in zip(dims[:-1], dims[1:]):
+        ldw = -(-K // 8) * 8
+        w = (torch.randn(N, ldw, generator=g) * 0.02).to(torch.bfloat16).to(DEV)[:, :K]
+        weights.append(fb.quantize_weight(w))
+    x0 = torch.randn(M, dims[0], generator=g).to(torch.bfloat16).to(DEV)
+    # separate calls
+    ref, h = [], x0
+    for mode, (q, s) in zip(modes, weights):
+        h = (fb.linear_w8a16 if mode == 0 else fb.linear_w8a8)(h, q, s)
+        ref.append(h)
+    # one sequence over fresh outputs
+    outs, jobs, h = [], [], x0
+    for mode, (q, s), r in zip(modes, weights, ref):
+        y = torch.full_like(r, 3.0)
+        jobs.append((mode, h, q, s, y))
+        outs.append(y)
+        h = y
+    for _ in range(2):                                  # repeated: rings and workspace reused
+        fb.linear_sequence(jobs)
+        torch.cuda.synchronize()
+        for r, y in zip(ref, outs):
+            assert torch.equal(y.view(torch.int16), r.view(torch.int16))
+    assert fb.read_device_error() == 0
