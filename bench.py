@@ -138,11 +138,20 @@ def oracle_sample_step(wl, wb, xb, n_rows):
 
 
 def calibrate_oracle_rows(wl, wb, xb, seconds: float) -> int:
-    t = time.perf_counter()
-    oracle_sample_step(wl, wb, xb, 128)
-    t1 = time.perf_counter() - t
-    blocks = max(1, min(-(-wl.N // 128), int(seconds / max(t1, 1e-6))))
-    return 128 * blocks
+    """Rows (a multiple of 128) for a sample step of about `seconds`: the
+    fixed cost (threads, the activation stage) and the cost per row are
+    fitted from two trials, 128 and 512 rows."""
+    nb = -(-wl.N // 128)
+    times = []
+    for rows in (128, min(512, 128 * nb)):
+        t = time.perf_counter()
+        oracle_sample_step(wl, wb, xb, rows)
+        times.append((rows, time.perf_counter() - t))
+    (r1, t1), (r2, t2) = times
+    per_row = (t2 - t1) / (r2 - r1) if r2 > r1 and t2 > t1 else t2 / r2
+    fixed = max(0.0, t1 - per_row * r1)
+    blocks = int((seconds - fixed) / max(per_row * 128, 1e-9))
+    return 128 * max(1, min(nb, blocks))
 
 
 def run_oracle(wl, wb, xb, seconds: float):
@@ -192,6 +201,24 @@ def reference_arm(args, wl):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ------------------------------------------------- replicas (N > 1 host logic)
+def replica_workload(wl, rank: int):
+    """The layer rank `rank` runs: its own seeded copy (replicas, no exchange)."""
+    from dataclasses import replace
+    return replace(wl, seed=wl.seed + rank)
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest `value` over all ranks (every rank calls this, in the same
+    order); the job's time is the slowest rank's."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -435,8 +462,7 @@ def main():
 
     M, K, N = wl.M, wl.K, wl.N
     # replicas: each rank its own seeded copy of the layer
-    from dataclasses import replace
-    wl_r = replace(wl, seed=wl.seed + rank)
+    wl_r = replica_workload(wl, rank)
     w_h = wl_r.weight_bf16()
     x_h = wl_r.x_bf16()
     w = w_h.to(dev)
@@ -493,10 +519,7 @@ def main():
     calls = ["quantize_weight", "dequantize", "linear_w8a16", "linear_w8a8"]
     per_call = {c: [ev[j].elapsed_time(ev[j + 1]) for ev in events] for j, c in enumerate(calls)}
     step_ms_total = sum(ev[0].elapsed_time(ev[4]) for ev in events)
-    t_local = torch.tensor([step_ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    step_ms_max = float(t_local.item()) / args.steps
+    step_ms_max = max_over_ranks(step_ms_total, world, dev) / args.steps
 
     flops_step = 2.0 * (2.0 * M * N * K)
     value = world * flops_step / (step_ms_max * 1e-3) / 1e12
@@ -607,11 +630,9 @@ def main():
         comp.wait_stream(h2d)
         e1.record(comp)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1) / e_steps], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        line["e2e"] = {"value": world * flops_step / (float(te.item()) * 1e-3) / 1e12,
-                       "unit": "TFLOP/s", "ms_per_step": float(te.item()), "steps": e_steps,
+        te = max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
+        line["e2e"] = {"value": world * flops_step / (te * 1e-3) / 1e12,
+                       "unit": "TFLOP/s", "ms_per_step": te, "steps": e_steps,
                        "h2d_bytes_per_step": 2 * N * K + 2 * M * K,
                        "d2h_bytes_per_step": 2 * 2 * M * N,
                        "pipelined": "steps overlap: upload of step i+1, compute of step i, "
