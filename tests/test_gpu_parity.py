@@ -282,20 +282,21 @@ def test_large_repeat_calls_are_deterministic(mode):
 @pytest.mark.gpu
 @pytest.mark.parametrize("M", [1, 16, 64, 128])
 def test_small_m_repeat_calls_are_deterministic(M):
-    """Stream-K at small token counts: two issuers, two expansion groups and
-    split tiles summed by the fix-up in a fixed order, so repeated calls must
-    be bit-identical (a race in any ring shows up as differing rows)."""
+    """Stream-K at small token counts (both linears): split tiles are summed
+    by the fix-up in a fixed order, so repeated calls must be bit-identical
+    (a race in any ring shows up as differing rows)."""
     K, N = 5120, 51200
     g = torch.Generator(device="cpu").manual_seed(11)
     w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
     x = torch.randn(M, K, generator=g).to(torch.bfloat16).to(DEV)
     q_d, s_d = fb.quantize_weight(w)
-    first = fb.linear_w8a16(x, q_d, s_d)
-    out = torch.empty_like(first)
-    for _ in range(5):
-        fb.linear_w8a16(x, q_d, s_d, out=out)
-        torch.cuda.synchronize()
-        assert torch.equal(out.view(torch.int16), first.view(torch.int16))
+    for f in (fb.linear_w8a16, fb.linear_w8a8):
+        first = f(x, q_d, s_d)
+        out = torch.empty_like(first)
+        for _ in range(5):
+            f(x, q_d, s_d, out=out)
+            torch.cuda.synchronize()
+            assert torch.equal(out.view(torch.int16), first.view(torch.int16))
     assert fb.read_device_error() == 0
 
 
