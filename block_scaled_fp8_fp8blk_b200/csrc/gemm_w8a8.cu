@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
                      const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ sx,
                      int64_t ldsx, const float* __restrict__ sw, uint16_t* __restrict__ y,
                      int64_t ldy, int M, int N, int n_tma, int KB, int mtiles, int ntiles_total,
-                     unsigned* __restrict__ err) {
+                     int a_bytes, unsigned* __restrict__ err) {
   using C = W8A8Cfg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
       // ------------------------------------------------- producers (A, B)
       const bool is_a = warp == 0;
       const CUtensorMap* map = is_a ? &tm_a : &tm_b;
-      const uint32_t bytes = is_a ? C::A_BYTES : C::B_BYTES;
+      const uint32_t bytes = is_a ? static_cast<uint32_t>(a_bytes) : C::B_BYTES;
       uint8_t* dst0 = smem + (is_a ? 0 : C::A_BYTES);
       tma_prefetch_map(map);
       // Launched as a programmatic dependent of the activation quantizer:
@@ -279,7 +279,12 @@ cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, c
                              bool after_act_quant) {
   using C = W8A8Cfg;
   CUtensorMap ta, tb, ty;
-  if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, K, M, ldqx, 128, C::BM))
+  // Fewer than BM tokens: load only the first round_up(M, 8) activation rows
+  // of a slab. The MMA still reads BM rows; the rows past those only reach
+  // output rows >= M, which are never stored.
+  const int64_t a_rows = M < C::BM ? round_up(M, 8) : C::BM;
+  if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, K, M, ldqx, 128,
+                    static_cast<uint32_t>(a_rows)))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, N, ldq, 128, C::BN))
     return cudaErrorInvalidValue;
@@ -324,7 +329,7 @@ cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, c
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, sx, ldsx, sw, y, ldy, static_cast<int>(M),
                             static_cast<int>(N), static_cast<int>(n_tma),
                             static_cast<int>(cdiv(K, 128)), static_cast<int>(mtiles),
-                            static_cast<int>(tiles), L.err);
+                            static_cast<int>(tiles), static_cast<int>(a_rows * 128), L.err);
 }
 
 }  // namespace fp8blk
