@@ -66,6 +66,22 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2_packed(uint64_t p) {
   return cvt_e4m3x2(hi, lo);
 }
 
+// Two BF16 values (low half -> low byte) -> the E4M3 codes of the bracket's
+// lower end; `diff` gets the bytes where the upper end gives another code
+// (a straddle, settled by the exact quotient).
+__device__ __forceinline__ uint32_t bracket2(uint32_t w2, const E4M3Divisor& dv, uint32_t& diff) {
+  const uint64_t f2 = pack_u32x2(w2 << 16, w2 & 0xFFFF0000u);
+  const uint32_t clo = cvt_e4m3x2_packed(fmul2(f2, dv.ylo2));
+  const uint32_t chi = cvt_e4m3x2_packed(fmul2(f2, dv.yhi2));
+  diff = clo ^ chi;
+  return clo;
+}
+
+// The exact codes of two BF16 values (two IEEE divisions).
+__device__ __forceinline__ uint32_t divide2(uint32_t w2, float d) {
+  return cvt_e4m3x2(__fdiv_rn(bf16_hi_to_f32(w2), d), __fdiv_rn(bf16_lo_to_f32(w2), d));
+}
+
 // Eight BF16 values -> eight E4M3 codes of RN_f32(v / d) (code i in byte i).
 // All 32 lanes of the warp must call this together. Element positions where
 // some lane's bracket straddles a decision point take the exact quotient
@@ -77,18 +93,12 @@ __device__ __forceinline__ uint2 encode8(const uint4& v, const E4M3Divisor& dv) 
   if (dv.exact) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      diff[i] = 0xFFFFu;
-      code[i] = 0u;
+      diff[i] = 0u;
+      code[i] = divide2(w[i], dv.d);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint64_t f2 = pack_u32x2(w[i] << 16, w[i] & 0xFFFF0000u);
-      const uint32_t clo = cvt_e4m3x2_packed(fmul2(f2, dv.ylo2));
-      const uint32_t chi = cvt_e4m3x2_packed(fmul2(f2, dv.yhi2));
-      diff[i] = clo ^ chi;
-      code[i] = clo;
-    }
+    for (int i = 0; i < 4; ++i) code[i] = bracket2(w[i], dv, diff[i]);
   }
   if (__any_sync(0xFFFFFFFFu, (diff[0] | diff[1] | diff[2] | diff[3]) != 0u)) {
 #pragma unroll
@@ -133,8 +143,11 @@ __device__ __forceinline__ void store8_codes(uint8_t* p, uint2 c, int valid) {
 // warps takes 16 rows of a block: lane l reads elements 4l..4l+3 of each row
 // (8-byte shared loads, conflict-free), the warps' maxima meet in shared
 // memory, and each lane then encodes its 64 values and writes 4 codes per row
-// (128 contiguous bytes per warp and row). Once the amax barrier is passed
-// every warp has read the stage, so thread 0 refills it right away.
+// (128 contiguous bytes per warp and row). Elements whose product bracket
+// straddles a decision point are settled after the block, each lane
+// re-reading its values from the stage, so a stage is refilled (by thread 0)
+// only once the next block's amax barrier shows every warp done with it:
+// two loads stay in flight per CTA.
 constexpr int kCvtStages = 3;
 constexpr int kCvtStageBytes = 128 * 128 * 2;
 constexpr size_t kCvtSmem = 128 + static_cast<size_t>(kCvtStages) * kCvtStageBytes;
@@ -189,7 +202,9 @@ __global__ void __launch_bounds__(256, 2) quantize_weight_kernel(
     }
     __syncthreads();
     if (abort_flag) break;
-    if (tid == 0) issue(i + kCvtStages);  // every warp has read this stage
+    // Every warp is done with the previous block's stage (its straddles
+    // included): refill it.
+    if (tid == 0 && i > 0) issue(i + kCvtStages - 1);
     m = red[i & 1][0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) m = max(m, red[i & 1][w]);
@@ -204,14 +219,22 @@ __global__ void __launch_bounds__(256, 2) quantize_weight_kernel(
     const int rows = static_cast<int>(N - n0 < 128 ? N - n0 : 128);
     const int cols = static_cast<int>(K - k0 < 128 ? K - k0 : 128);
     const int col = 4 * lane;
+    // Provisional codes from the bracket's lower end, with one bit per row
+    // pair in which this lane saw a straddle (every pair when d is too small
+    // for the bracket).
+    uint32_t straddled = dv.exact ? 0xFFu : 0u;
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
-      // rows 2g and 2g + 1 of this warp's 16: every lane encodes (warp vote inside)
-      const uint2 c = encode8(make_uint4(v[2 * g].x, v[2 * g].y, v[2 * g + 1].x, v[2 * g + 1].y), dv);
+      // rows 2g and 2g + 1 of this warp's 16, four columns each
+      const uint32_t w4[4] = {v[2 * g].x, v[2 * g].y, v[2 * g + 1].x, v[2 * g + 1].y};
+      uint32_t code[4], diff[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) code[k] = bracket2(w4[k], dv, diff[k]);
+      straddled |= ((diff[0] | diff[1] | diff[2] | diff[3]) != 0u ? 1u : 0u) << g;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int r = warp * 16 + 2 * g + h;
-        const uint32_t codes = h ? c.y : c.x;
+        const uint32_t codes = code[2 * h] | (code[2 * h + 1] << 16);
         if (r < rows && col < cols) {
           uint8_t* dst = q + (n0 + r) * ldq + k0 + col;
           if (col + 4 <= cols) {
@@ -222,10 +245,42 @@ __global__ void __launch_bounds__(256, 2) quantize_weight_kernel(
         }
       }
     }
+    // Straddles (rare): each lane re-reads its row pairs that had one from
+    // the stage (still resident: it is refilled only after the next amax
+    // barrier) and writes the exact quotient's code over the provisional one.
+    while (straddled != 0u) {
+      const int g = __ffs(straddled) - 1;
+      straddled &= straddled - 1u;
+      const uint8_t* src = smem + st * kCvtStageBytes + (warp * 16 + 2 * g) * 256 + lane * 8;
+      const uint2 a = *reinterpret_cast<const uint2*>(src);
+      const uint2 c = *reinterpret_cast<const uint2*>(src + 256);
+      const uint32_t w4[4] = {a.x, a.y, c.x, c.y};
+      uint32_t elems = 0;  // bit 2k + h: half h of word k straddles
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t diff;
+        bracket2(w4[k], dv, diff);
+        if (dv.exact) diff = 0xFFFFu;
+        elems |= (((diff & 0xFFu) != 0u ? 1u : 0u) | ((diff >> 8) != 0u ? 2u : 0u)) << (2 * k);
+      }
+      // one element per lane and pass: the lanes' divisions run side by side
+      while (elems != 0u) {
+        const int t = __ffs(elems) - 1;
+        elems &= elems - 1u;
+        const int k = t >> 1;
+        const uint32_t wd = (k & 2) ? ((k & 1) ? w4[3] : w4[2]) : ((k & 1) ? w4[1] : w4[0]);
+        const float x = (t & 1) ? bf16_hi_to_f32(wd) : bf16_lo_to_f32(wd);
+        const uint32_t code = cvt_e4m3x2(0.0f, __fdiv_rn(x, dv.d)) & 0xFFu;
+        const int r = warp * 16 + 2 * g + (k >> 1), cc = col + 2 * (k & 1) + (t & 1);
+        if (r < rows && cc < cols) q[(n0 + r) * ldq + k0 + cc] = static_cast<uint8_t>(code);
+      }
+    }
   }
   // After a time-out, the loads still in flight land before the CTA exits.
   if (tid == 0 && abort_flag) {
-    for (int k = i; k < i + kCvtStages; ++k) {
+    // issued so far: blocks 0 .. max(kCvtStages - 1, i + kCvtStages - 2)
+    const int last = i + kCvtStages - 2 > kCvtStages - 1 ? i + kCvtStages - 2 : kCvtStages - 1;
+    for (int k = i; k <= last; ++k) {
       const int b = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
       if (b < nblocks) mbar_wait(&full[k % kCvtStages], static_cast<uint32_t>((k / kCvtStages) & 1), err, kErrWaitLoad);
     }

@@ -112,6 +112,59 @@ def test_quantize_zero_blocks_and_signs():
     assert np.array_equal(s_d.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
+def _e4m3_midpoints(limit: float) -> np.ndarray:
+    """Every positive value halfway between two neighbouring E4M3 values, up to limit."""
+    sub = (2 * np.arange(7) + 1) * 2.0 ** -10
+    norm = [(1 + (2 * j + 1) / 16) * 2.0 ** e for e in range(-6, 9) for j in range(8)]
+    m = np.concatenate([sub, np.array(norm)])
+    return m[m <= limit]
+
+
+def test_quantize_tie_heavy_blocks():
+    """Blocks whose quotients v / s sit exactly on E4M3 decision points (the
+    product bracket straddles there and the exact quotient decides, ties to
+    even): per warp of 16 rows none, a few, 31 / 33 / 40 / 63 / 64 / 65 of
+    them, and whole blocks of them (more than a warp settles in one round),
+    with ragged edges."""
+    rng = np.random.default_rng(77)
+    N, K = 200, 300                       # block row 1 has 72 rows, block column 2 has 44
+    mids = _e4m3_midpoints(432.0)
+    # ordinary values: 8 significant bits (lowest BF16 fraction bit set), never a tie at s = 1 or 2
+    base = synth.bf16_bits(synth.to_bf16(rng.standard_normal((N, K)).astype(np.float32) * 60.0))
+    base = base | np.uint16(1)
+    w = (base.astype(np.uint32) << 16).view(np.float32).copy()
+    np.clip(w, -440.0, 440.0, out=w)
+    w = synth.bf16_bits(synth.to_bf16(w)) | np.uint16(1)
+    w = (w.astype(np.uint32) << 16).view(np.float32).copy()
+
+    def ties(n):
+        return rng.choice(mids, n) * rng.choice([-1.0, 1.0], n)
+
+    # block (0, 0): amax 448 (s = 1), warps with 0, 5, 31, 33, 40, 63, 64, 65 ties
+    for wi, n in enumerate([0, 5, 31, 33, 40, 63, 64, 65]):
+        pos = rng.choice(16 * 128, n, replace=False)
+        w[16 * wi + pos // 128, pos % 128] = ties(n)
+    w[0, 0] = 448.0
+    # block (0, 1): every element a tie, amax 896 (s = 2)
+    w[:128, 128:256] = 2.0 * ties(128 * 128).reshape(128, 128)
+    w[77, 200] = -896.0
+    # block (0, 2) (44 columns): ties in the last columns, amax 448
+    w[:128, 290:300] = ties(1280).reshape(128, 10)
+    w[3, 256] = 448.0
+    # block (1, 0) (72 rows): ties on the last rows
+    w[190:200, :128] = ties(1280).reshape(10, 128)
+    w[128, 5] = 448.0
+    # block (1, 2) (72 x 44): every element a tie, amax 448
+    w[128:200, 256:300] = ties(72 * 44).reshape(72, 44)
+    w[199, 299] = 448.0
+    wb = synth.bf16_bits(synth.to_bf16(w))
+    assert np.array_equal((wb.astype(np.uint32) << 16).view(np.float32), w), "values must be BF16"
+    q_ref, s_ref = oracle.quantize_weight(wb)
+    q_d, s_d = fb.quantize_weight(to_dev_bf16(wb))
+    assert np.array_equal(s_d.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(u8(q_d), q_ref)
+
+
 def test_quantize_every_bf16_value():
     allb = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
     vals = (allb.astype(np.uint32) << 16).view(np.float32)
@@ -441,4 +494,51 @@ def test_linear_sequence_matches_separate_calls(M):
         torch.cuda.synchronize()
         for r, y in zip(ref, outs):
             assert torch.equal(y.view(torch.int16), r.view(torch.int16))
+    assert fb.read_device_error() == 0
+
+
+@pytest.mark.gpu
+def test_sequence_and_streaming_edge_jobs():
+    """Jobs with K = 0 (y = 0) and N = 0 (nothing) inside a sequence and a
+    streamed run, between ordinary jobs."""
+    g = torch.Generator(device="cpu").manual_seed(51)
+    w = (torch.randn(384, 256, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
+    q, s = fb.quantize_weight(w)
+    x = torch.randn(64, 256, generator=g).to(torch.bfloat16).to(DEV)
+    ref = fb.linear_w8a16(x, q, s)
+    x0 = torch.zeros((64, 0), dtype=torch.bfloat16, device=DEV)
+    q0 = torch.zeros((384, 0), dtype=torch.uint8, device=DEV)
+    s0 = torch.zeros((3, 1), dtype=torch.float32, device=DEV)
+    qn = torch.zeros((0, 256), dtype=torch.uint8, device=DEV)
+    sn = torch.zeros((1, 2), dtype=torch.float32, device=DEV)
+    # sequence
+    y1, y2 = torch.full_like(ref, 5.0), torch.full_like(ref, 5.0)
+    yk0 = torch.full_like(ref, 5.0)
+    yn0 = torch.empty((64, 0), dtype=torch.bfloat16, device=DEV)
+    fb.linear_sequence([(0, x, q, s, y1), (1, x0, q0, s0, yk0), (0, x, qn, sn, yn0), (0, x, q, s, y2)])
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(y2.view(torch.int16), ref.view(torch.int16))
+    assert torch.all(yk0 == 0)
+    # streaming (host weights; the K = 0 job copies nothing)
+    qh = torch.empty(q.shape, dtype=torch.uint8, pin_memory=True)
+    qh.copy_(q)
+    sh = s.cpu().pin_memory()
+    q0h = torch.empty((384, 0), dtype=torch.uint8, pin_memory=True)
+    s0h = torch.zeros((3, 1), dtype=torch.float32).pin_memory()
+    y3, y4 = torch.full_like(ref, 5.0), torch.full_like(ref, 5.0)
+    yk1 = torch.full_like(ref, 5.0)
+    slot = -(-fb.stream_slot_bytes(384, 256, 256) // 256) * 256
+    slots = torch.empty(2 * slot, dtype=torch.uint8, device=DEV)
+    ws = torch.empty(fb.workspace_size(0, 64, 384, 256), dtype=torch.uint8, device=DEV)
+    compute, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    events = [torch.cuda.Event() for _ in range(4)]
+    compute.wait_stream(torch.cuda.current_stream())
+    fb.streamed_linears([(0, qh, sh, x, y3), (0, q0h, s0h, x0, yk1), (0, qh, sh, x, y4)],
+                        slots, slot, 2, ws, compute, copy, events)
+    torch.cuda.current_stream().wait_stream(compute)
+    torch.cuda.synchronize()
+    assert torch.equal(y3.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(y4.view(torch.int16), ref.view(torch.int16))
+    assert torch.all(yk1 == 0)
     assert fb.read_device_error() == 0
