@@ -230,7 +230,8 @@ def traffic_for(kernel_file: str, key: str):
         with open(path) as f:
             rec = json.load(f).get(key)
         src = os.path.join(ROOT, "block_scaled_fp8_fp8blk_b200", "csrc", kernel_file)
-        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
         if rec and rec.get("source_sha256_16") == digest:
             return rec.get("dram_bytes_per_launch")
     except (OSError, ValueError):

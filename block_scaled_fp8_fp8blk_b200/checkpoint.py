@@ -176,6 +176,15 @@ def save_checkpoint(out_dir: str, tensors: dict, config: dict | None = None,
     return index
 
 
+def _read_config(directory: str) -> dict:
+    """config.json of a checkpoint directory, or {} when it has none."""
+    path = os.path.join(directory, "config.json")
+    if not os.path.exists(path):
+        return {}
+    with open(path) as f:
+        return json.load(f)
+
+
 def load_checkpoint(in_dir: str, names: Iterable[str] | None = None) -> tuple[dict, dict]:
     """Reads a checkpoint written by :func:`save_checkpoint` (or any
     directory with the same index): returns (CPU tensors, config)."""
@@ -189,9 +198,7 @@ def load_checkpoint(in_dir: str, names: Iterable[str] | None = None) -> tuple[di
     out = {}
     for fname, ns in by_file.items():
         out.update(read_safetensors(os.path.join(in_dir, fname), ns))
-    cfg_path = os.path.join(in_dir, "config.json")
-    config = json.load(open(cfg_path)) if os.path.exists(cfg_path) else {}
-    return out, config
+    return out, _read_config(in_dir)
 
 
 def convert_checkpoint(src_dir: str, dst_dir: str, is_linear: Callable = default_is_linear,
@@ -208,9 +215,7 @@ def convert_checkpoint(src_dir: str, dst_dir: str, is_linear: Callable = default
     for fname in files:
         converted.update(quantize_state_dict(read_safetensors(os.path.join(src_dir, fname)),
                                              is_linear))
-    cfg_path = os.path.join(src_dir, "config.json")
-    config = json.load(open(cfg_path)) if os.path.exists(cfg_path) else {}
-    return save_checkpoint(dst_dir, converted, config, max_shard_bytes)
+    return save_checkpoint(dst_dir, converted, _read_config(src_dir), max_shard_bytes)
 
 
 def linear_weights(tensors: dict, name: str, device: str | torch.device = "cuda",
