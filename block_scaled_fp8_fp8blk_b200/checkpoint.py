@@ -119,15 +119,16 @@ def quantize_state_dict(state: dict, is_linear: Callable = default_is_linear,
     """Converts every linear weight of ``state`` with the GPU converter
     (``fp8blk_quantize_weight``): ``<p>.weight`` -> E4M3 codes [N, K] (dtype
     float8_e4m3fn, CPU) + ``<p>.weight_scale_inv`` float32; other tensors are
-    returned unchanged. Raises without a CUDA device (no CPU path)."""
+    returned unchanged. Raises without a CUDA device when there is a linear
+    to convert (there is no CPU path)."""
     import block_scaled_fp8_fp8blk_b200 as fb
-    if not torch.cuda.is_available():
-        raise RuntimeError("quantize_state_dict needs a CUDA device (the converter is a GPU kernel)")
     out = {}
     for name, t in state.items():
         if not is_linear(name, t):
             out[name] = t
             continue
+        if not torch.cuda.is_available():
+            raise RuntimeError("quantize_state_dict needs a CUDA device (the converter is a GPU kernel)")
         w = t.detach().to(device=device, dtype=torch.bfloat16).contiguous()
         N, K = w.shape
         ldw = -(-K // 8) * 8

@@ -124,3 +124,26 @@ def test_quantize_state_dict_needs_a_gpu(monkeypatch):
     monkeypatch.setattr(torch.cuda, "is_available", lambda: False)
     with pytest.raises(RuntimeError, match="CUDA"):
         ck.quantize_state_dict({"l.weight": torch.ones(4, 4)})
+
+
+def test_convert_checkpoint_without_linears_passes_through(tmp_path, monkeypatch):
+    """With nothing to quantize no GPU is needed: the converter re-shards the
+    tensors unchanged and keeps the source config (no quantization_config,
+    since no tensor is E4M3)."""
+    monkeypatch.setattr(torch.cuda, "is_available", lambda: False)
+    g = torch.Generator().manual_seed(9)
+    src_t = {"model.norm.weight": torch.randn(64, generator=g).to(torch.bfloat16),
+             "model.embed_tokens.weight": torch.randn(40, 16, generator=g).to(torch.bfloat16),
+             "model.layers.0.mlp.up_proj.weight": torch.randn(8, 8, generator=g).to(torch.bfloat16)}
+    src = str(tmp_path / "src")
+    ck.save_checkpoint(src, src_t, {"model_type": "toy", "hidden_size": 16}, max_shard_bytes=200)
+    dst = str(tmp_path / "dst")
+    idx = ck.convert_checkpoint(src, dst, is_linear=lambda n, t: False, max_shard_bytes=10**6)
+    assert set(idx["weight_map"]) == set(src_t)
+    assert len(set(idx["weight_map"].values())) == 1          # one shard at the larger limit
+    back, cfg = ck.load_checkpoint(dst)
+    assert cfg == {"model_type": "toy", "hidden_size": 16}
+    for k, v in src_t.items():
+        same(back[k], v)
+    with pytest.raises(RuntimeError, match="CUDA"):           # a linear still needs the GPU
+        ck.convert_checkpoint(src, str(tmp_path / "dst2"))
