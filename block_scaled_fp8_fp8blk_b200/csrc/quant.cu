@@ -148,6 +148,40 @@ __device__ __forceinline__ void store8_codes(uint8_t* p, uint2 c, int valid) {
 // re-reading its values from the stage, so a stage is refilled (by thread 0)
 // only once the next block's amax barrier shows every warp done with it:
 // two loads stay in flight per CTA.
+// A warp's 16 rows of one block: codes of the bracket's lower end stored
+// row by row (4 per lane), returning one bit per row pair with a straddle.
+// Interior blocks store without bounds checks; otherwise rows_left and
+// cols_left are the rows and columns of this lane's part inside the matrix.
+template <bool Interior>
+__device__ __forceinline__ uint32_t encode_rows(const uint2 (&v)[16], const E4M3Divisor& dv,
+                                                uint8_t* dst, int64_t ldq, int rows_left,
+                                                int cols_left) {
+  uint32_t straddled = 0u;
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    const uint32_t w4[4] = {v[2 * g].x, v[2 * g].y, v[2 * g + 1].x, v[2 * g + 1].y};
+    uint32_t code[4], diff[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) code[k] = bracket2(w4[k], dv, diff[k]);
+    straddled |= ((diff[0] | diff[1] | diff[2] | diff[3]) != 0u ? 1u : 0u) << g;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t codes = code[2 * h] | (code[2 * h + 1] << 16);
+      if (Interior) {
+        __stcs(reinterpret_cast<unsigned int*>(dst), codes);
+      } else if (2 * g + h < rows_left && cols_left > 0) {
+        if (cols_left >= 4) {
+          __stcs(reinterpret_cast<unsigned int*>(dst), codes);
+        } else {
+          for (int t = 0; t < cols_left; ++t) dst[t] = static_cast<uint8_t>(codes >> (8 * t));
+        }
+      }
+      dst += ldq;
+    }
+  }
+  return straddled;
+}
+
 constexpr int kCvtStages = 3;
 constexpr int kCvtStageBytes = 128 * 128 * 2;
 constexpr size_t kCvtSmem = 128 + static_cast<size_t>(kCvtStages) * kCvtStageBytes;
@@ -223,28 +257,11 @@ __global__ void __launch_bounds__(256, 2) quantize_weight_kernel(
     // pair in which this lane saw a straddle (every pair when d is too small
     // for the bracket).
     uint32_t straddled = dv.exact ? 0xFFu : 0u;
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      // rows 2g and 2g + 1 of this warp's 16, four columns each
-      const uint32_t w4[4] = {v[2 * g].x, v[2 * g].y, v[2 * g + 1].x, v[2 * g + 1].y};
-      uint32_t code[4], diff[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) code[k] = bracket2(w4[k], dv, diff[k]);
-      straddled |= ((diff[0] | diff[1] | diff[2] | diff[3]) != 0u ? 1u : 0u) << g;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = warp * 16 + 2 * g + h;
-        const uint32_t codes = code[2 * h] | (code[2 * h + 1] << 16);
-        if (r < rows && col < cols) {
-          uint8_t* dst = q + (n0 + r) * ldq + k0 + col;
-          if (col + 4 <= cols) {
-            __stcs(reinterpret_cast<unsigned int*>(dst), codes);
-          } else {
-            for (int t = 0; t < cols - col; ++t) dst[t] = static_cast<uint8_t>(codes >> (8 * t));
-          }
-        }
-      }
-    }
+    uint8_t* dst0 = q + (n0 + warp * 16) * ldq + k0 + col;
+    if (rows == 128 && cols == 128)
+      straddled |= encode_rows<true>(v, dv, dst0, ldq, 16, 4);
+    else
+      straddled |= encode_rows<false>(v, dv, dst0, ldq, rows - warp * 16, cols - col);
     // Straddles (rare): each lane re-reads its row pairs that had one from
     // the stage (still resident: it is refilled only after the next amax
     // barrier) and writes the exact quotient's code over the provisional one.
