@@ -55,3 +55,50 @@ def oracle_refs(wl, wb: np.ndarray, xb: np.ndarray, rows=None):
     r16 = oracle.linear_w8a16(xb, q, s, wl.N, wl.K, rows=rows)
     r8 = oracle.linear_w8a8(qx, sx, q, s, wl.N, wl.K, rows=rows)
     return q, s, r16, r8, qx, sx
+
+
+def e4m3_midpoints(limit: float) -> np.ndarray:
+    """Every positive value halfway between two neighbouring E4M3 values, up to limit."""
+    sub = (2 * np.arange(7) + 1) * 2.0 ** -10
+    norm = [(1 + (2 * j + 1) / 16) * 2.0 ** e for e in range(-6, 9) for j in range(8)]
+    m = np.concatenate([sub, np.array(norm)])
+    return m[m <= limit]
+
+
+def tie_heavy_weight() -> np.ndarray:
+    """BF16 bits of a 200 x 300 weight whose quotients v / s sit exactly on
+    E4M3 decision points in controlled numbers. Block (0, 0) has amax 448
+    (s = 1) and per warp of 16 rows 0, 5, 31, 33, 40, 63, 64 or 65 ties.
+    Block (0, 1) is all ties at amax 896 (s = 2). Ties also sit on the last
+    columns of block (0, 2), which is 44 columns wide, and on the last rows
+    of block (1, 0), which is 72 rows high. Block (1, 2) is all ties. All
+    other values have 8 significant bits, so they are never a tie at
+    s = 1 or 2."""
+    rng = np.random.default_rng(77)
+    N, K = 200, 300
+    mids = e4m3_midpoints(432.0)
+    base = synth.bf16_bits(synth.to_bf16(rng.standard_normal((N, K)).astype(np.float32) * 60.0))
+    base = base | np.uint16(1)
+    w = (base.astype(np.uint32) << 16).view(np.float32).copy()
+    np.clip(w, -440.0, 440.0, out=w)
+    w = synth.bf16_bits(synth.to_bf16(w)) | np.uint16(1)
+    w = (w.astype(np.uint32) << 16).view(np.float32).copy()
+
+    def ties(n):
+        return rng.choice(mids, n) * rng.choice([-1.0, 1.0], n)
+
+    for wi, n in enumerate([0, 5, 31, 33, 40, 63, 64, 65]):
+        pos = rng.choice(16 * 128, n, replace=False)
+        w[16 * wi + pos // 128, pos % 128] = ties(n)
+    w[0, 0] = 448.0
+    w[:128, 128:256] = 2.0 * ties(128 * 128).reshape(128, 128)
+    w[77, 200] = -896.0
+    w[:128, 290:300] = ties(1280).reshape(128, 10)
+    w[3, 256] = 448.0
+    w[190:200, :128] = ties(1280).reshape(10, 128)
+    w[128, 5] = 448.0
+    w[128:200, 256:300] = ties(72 * 44).reshape(72, 44)
+    w[199, 299] = 448.0
+    wb = synth.bf16_bits(synth.to_bf16(w))
+    assert np.array_equal((wb.astype(np.uint32) << 16).view(np.float32), w), "values must be BF16"
+    return wb

@@ -13,7 +13,7 @@ import torch
 import block_scaled_fp8_fp8blk_b200 as fb
 import oracle
 from block_scaled_fp8_fp8blk_b200 import synth, workloads as W
-from helpers import bf16_bits, bf16_to_f64, check_linear
+from helpers import bf16_bits, bf16_to_f64, check_linear, tie_heavy_weight
 
 pytestmark = pytest.mark.gpu
 
@@ -112,53 +112,12 @@ def test_quantize_zero_blocks_and_signs():
     assert np.array_equal(s_d.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
-def _e4m3_midpoints(limit: float) -> np.ndarray:
-    """Every positive value halfway between two neighbouring E4M3 values, up to limit."""
-    sub = (2 * np.arange(7) + 1) * 2.0 ** -10
-    norm = [(1 + (2 * j + 1) / 16) * 2.0 ** e for e in range(-6, 9) for j in range(8)]
-    m = np.concatenate([sub, np.array(norm)])
-    return m[m <= limit]
-
-
 def test_quantize_tie_heavy_blocks():
     """Blocks whose quotients v / s sit exactly on E4M3 decision points (the
     product bracket straddles there and the exact quotient decides, ties to
     even): per warp of 16 rows none, a few, 31 / 33 / 40 / 63 / 64 / 65 of
-    them, and whole blocks of them (more than a warp settles in one round),
-    with ragged edges."""
-    rng = np.random.default_rng(77)
-    N, K = 200, 300                       # block row 1 has 72 rows, block column 2 has 44
-    mids = _e4m3_midpoints(432.0)
-    # ordinary values: 8 significant bits (lowest BF16 fraction bit set), never a tie at s = 1 or 2
-    base = synth.bf16_bits(synth.to_bf16(rng.standard_normal((N, K)).astype(np.float32) * 60.0))
-    base = base | np.uint16(1)
-    w = (base.astype(np.uint32) << 16).view(np.float32).copy()
-    np.clip(w, -440.0, 440.0, out=w)
-    w = synth.bf16_bits(synth.to_bf16(w)) | np.uint16(1)
-    w = (w.astype(np.uint32) << 16).view(np.float32).copy()
-
-    def ties(n):
-        return rng.choice(mids, n) * rng.choice([-1.0, 1.0], n)
-
-    # block (0, 0): amax 448 (s = 1), warps with 0, 5, 31, 33, 40, 63, 64, 65 ties
-    for wi, n in enumerate([0, 5, 31, 33, 40, 63, 64, 65]):
-        pos = rng.choice(16 * 128, n, replace=False)
-        w[16 * wi + pos // 128, pos % 128] = ties(n)
-    w[0, 0] = 448.0
-    # block (0, 1): every element a tie, amax 896 (s = 2)
-    w[:128, 128:256] = 2.0 * ties(128 * 128).reshape(128, 128)
-    w[77, 200] = -896.0
-    # block (0, 2) (44 columns): ties in the last columns, amax 448
-    w[:128, 290:300] = ties(1280).reshape(128, 10)
-    w[3, 256] = 448.0
-    # block (1, 0) (72 rows): ties on the last rows
-    w[190:200, :128] = ties(1280).reshape(10, 128)
-    w[128, 5] = 448.0
-    # block (1, 2) (72 x 44): every element a tie, amax 448
-    w[128:200, 256:300] = ties(72 * 44).reshape(72, 44)
-    w[199, 299] = 448.0
-    wb = synth.bf16_bits(synth.to_bf16(w))
-    assert np.array_equal((wb.astype(np.uint32) << 16).view(np.float32), w), "values must be BF16"
+    them, and whole blocks of them, with ragged edges."""
+    wb = tie_heavy_weight()
     q_ref, s_ref = oracle.quantize_weight(wb)
     q_d, s_d = fb.quantize_weight(to_dev_bf16(wb))
     assert np.array_equal(s_d.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))

@@ -12,6 +12,7 @@ import oracle
 from block_scaled_fp8_fp8blk_b200 import synth
 from block_scaled_fp8_fp8blk_b200.workloads import RAGGED, TINY, Workload
 from conftest import read_golden
+from helpers import e4m3_midpoints, tie_heavy_weight
 
 TORCH_E4M3 = torch.float8_e4m3fn
 
@@ -85,6 +86,24 @@ def test_codes_match_torch_division_and_cast(wl, weights):
     ratio = (torch.from_numpy(wf) / torch.from_numpy(np.ascontiguousarray(sb))).numpy()
     assert np.abs(ratio).max() < 464
     assert np.array_equal(q, torch_codes(ratio))
+
+
+def test_tie_heavy_blocks_round_to_even():
+    """Quotients exactly on E4M3 decision points, whole blocks of them and a
+    few per warp's rows, with ragged edges: the codes equal torch's float32
+    division and float8 cast, and every tie took the even code."""
+    wb = tie_heavy_weight()
+    q, s = oracle.quantize_weight(wb)
+    N, K = wb.shape
+    wf = f32_from_bf16(wb)
+    assert np.array_equal(s, block_amax(wf, N, K) / np.float32(448.0))
+    sb = broadcast(s, N, K)
+    ratio = (torch.from_numpy(wf) / torch.from_numpy(np.ascontiguousarray(sb))).numpy()
+    assert np.array_equal(q, torch_codes(ratio))
+    mids = set(e4m3_midpoints(464.0).tolist())
+    tie = np.vectorize(lambda r: abs(float(r)) in mids)(ratio)
+    assert tie.sum() > 20000                      # the blocks really are tie-heavy
+    assert np.all((q[tie] & 1) == 0)              # ties to even: the code's last bit is 0
 
 
 def test_block_max_code_is_448(wl, weights):
