@@ -40,6 +40,7 @@ def _load():
             "orc_e4m3_encode_array": (None, [_p, _i64, _p]),
             "orc_bf16_rne_array": (None, [_p, _i64, _p]),
             "orc_crosscheck_encoders": (_i64, [_u64, _u64, _int]),
+            "orc_crosscheck_encoders_planted": (_i64, [_u64, _u64, _u64, _int]),
             "orc_count_code_mismatches": (_i64, [_u64, _i64, _p, _int]),
             "orc_quantize_weight": (None, [_p, _i64, _i64, _i64, _p, _i64, _p, _int]),
             "orc_dequantize": (None, [_p, _i64, _p, _i64, _i64, _p, _i64, _int]),
@@ -97,6 +98,12 @@ def bf16_rne(v) -> np.ndarray:
 
 def crosscheck_encoders(lo: int, hi: int, nthreads: int | None = None) -> int:
     return int(_load().orc_crosscheck_encoders(lo, hi, nthreads or threads()))
+
+
+def crosscheck_encoders_planted(lo: int, hi: int, planted: int, nthreads: int | None = None) -> int:
+    """Test hook: the cross-check with the bit-field encoder's code at bit
+    pattern `planted` deliberately wrong (lowest bit flipped)."""
+    return int(_load().orc_crosscheck_encoders_planted(lo, hi, planted, nthreads or threads()))
 
 
 def count_code_mismatches(lo: int, codes: np.ndarray, nthreads: int | None = None) -> int:

@@ -193,7 +193,11 @@ void orc_bf16_rne_array(const float* v, int64_t n, uint16_t* out) {
 }
 
 // Number of float bit patterns in [lo, hi) where the two encoders disagree.
-int64_t orc_crosscheck_encoders(uint64_t lo, uint64_t hi, int nthreads) {
+// `planted` is a test hook: at that bit pattern the bit-field encoder's code
+// is taken with its lowest bit flipped, so a test can check that one planted
+// disagreement is counted exactly once (no bit pattern equals the default,
+// which is above 2^32).
+static int64_t crosscheck_encoders(uint64_t lo, uint64_t hi, uint64_t planted, int nthreads) {
   if (hi <= lo) return 0;
   const uint64_t chunk = 1ull << 20;
   const int64_t nchunks = int64_t((hi - lo + chunk - 1) / chunk);
@@ -205,13 +209,23 @@ int64_t orc_crosscheck_encoders(uint64_t lo, uint64_t hi, int nthreads) {
       uint32_t bits = uint32_t(u);
       float f;
       std::memcpy(&f, &bits, 4);
-      cnt += e4m3_encode_search(f) != e4m3_encode_fields(f);
+      uint8_t by_fields = e4m3_encode_fields(f);
+      if (u == planted) by_fields ^= 1u;
+      cnt += e4m3_encode_search(f) != by_fields;
     }
     bad[size_t(ci)] = cnt;
   });
   int64_t total = 0;
   for (auto c : bad) total += c;
   return total;
+}
+
+int64_t orc_crosscheck_encoders(uint64_t lo, uint64_t hi, int nthreads) {
+  return crosscheck_encoders(lo, hi, ~0ull, nthreads);
+}
+
+int64_t orc_crosscheck_encoders_planted(uint64_t lo, uint64_t hi, uint64_t planted, int nthreads) {
+  return crosscheck_encoders(lo, hi, planted, nthreads);
 }
 
 // Mismatches between given codes and the oracle's encoding of the float bit

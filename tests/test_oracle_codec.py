@@ -127,3 +127,80 @@ def test_bf16_rne_is_nearest_ties_even():
     assert np.all(d_r == d_o)
     tie = np.abs(lo - x) == np.abs(hi - x)
     assert np.all(((out[tie] >> 16) & 1) == 0)
+
+
+# ------------------------------------------- the two whole-range checkers
+# Both checkers return a count that the exhaustive tests require to be 0. A
+# count that came out 0 for a wrong reason (a chunk skipped, a loop bound off
+# by one, threads that never ran) would turn those tests into no-ops, so the
+# counts themselves are pinned here: a planted error is counted exactly once
+# wherever it sits (first or last pattern, either side of a chunk boundary,
+# in a short last chunk) and with any number of threads.
+CHUNK = 1 << 20
+
+
+def _planted_positions(n):
+    return sorted({0, 1, CHUNK - 1, CHUNK, CHUNK + 1, 2 * CHUNK - 1, 2 * CHUNK, n // 2, n - 2, n - 1})
+
+
+def test_code_mismatch_count_against_torch_codes_and_planted_errors():
+    lo = 0x3E000000 - 3                          # floats just below and above 0.125
+    n = 2 * CHUNK + 123                           # three chunks, the last one short
+    v = (np.arange(n, dtype=np.uint64) + lo).astype(np.uint32).view(np.float32)
+    assert np.all(np.abs(v) < 448)                # torch's cast saturates nothing here
+    codes = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy().copy()
+    for nthreads in (1, 3, 16):
+        assert oracle.count_code_mismatches(lo, codes, nthreads) == 0
+    for pos in _planted_positions(n):
+        bad = codes.copy()
+        bad[pos] ^= 0x01
+        for nthreads in (1, 3, 16):
+            assert oracle.count_code_mismatches(lo, bad, nthreads) == 1, (pos, nthreads)
+    bad = codes.copy()
+    planted = _planted_positions(n)
+    bad[planted] ^= 0x40
+    assert oracle.count_code_mismatches(lo, bad) == len(planted)
+    # a code array shifted by one pattern disagrees wherever neighbours differ
+    shifted = np.roll(codes, 1)
+    want = int(np.count_nonzero(shifted != codes))
+    assert want > 0 and oracle.count_code_mismatches(lo, shifted) == want
+
+
+def test_bit_field_encoder_matches_torch_on_a_range():
+    # the encoder the device codec is counted against, checked against torch's
+    # cast on every pattern of a range that crosses the E4M3 subnormal/normal
+    # boundary (2^-6) and a few binades of normals
+    lo, hi = 0x3C000000, 0x3C000000 + (1 << 24)  # 2^-7 up to 2^-5
+    v = np.arange(lo, hi, 37, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode_fields(float(f)) for f in v[::64]], dtype=np.uint8)
+    assert np.array_equal(got, ref[::64])
+
+
+def test_encoder_crosscheck_counts_a_planted_disagreement():
+    lo = 0x43D00000 - 5                          # around 416 .. saturation
+    hi = lo + 2 * CHUNK + 77
+    assert oracle.crosscheck_encoders(lo, hi) == 0
+    for off in _planted_positions(hi - lo):
+        for nthreads in (1, 4, 16):
+            assert oracle.crosscheck_encoders_planted(lo, hi, lo + off, nthreads) == 1, (off, nthreads)
+    # a plant outside the range is not counted
+    assert oracle.crosscheck_encoders_planted(lo, hi, lo - 1, 4) == 0
+    assert oracle.crosscheck_encoders_planted(lo, hi, hi, 4) == 0
+    # the top of the 32-bit range (the last chunk ends at 2^32 exactly)
+    top = (1 << 32) - CHUNK - 9
+    assert oracle.crosscheck_encoders_planted(top, 1 << 32, (1 << 32) - 1, 8) == 1
+    assert oracle.crosscheck_encoders_planted(top, 1 << 32, top, 8) == 1
+
+
+def test_encoder_crosscheck_equals_a_count_one_pattern_at_a_time():
+    # brute force over a small range: the count equals the number of patterns
+    # where the two single-value encoders differ (here none, and the planted one)
+    lo, hi = 0x3A7FFFF0, 0x3A800010              # around 2^-10, where codes underflow to 0
+    diffs = 0
+    for u in range(lo, hi):
+        f = f32(u)
+        diffs += int(oracle.e4m3_encode(np.array([f], np.float32))[0] != oracle.e4m3_encode_fields(f))
+    assert diffs == 0
+    assert oracle.crosscheck_encoders(lo, hi, 1) == diffs
+    assert oracle.crosscheck_encoders_planted(lo, hi, lo + 7, 1) == diffs + 1
