@@ -7,8 +7,13 @@ on the headline layer (M=512 tokens, K=5120, N=25600, the largest linear of a
   linear_w8a16 (x BF16 . dequant(W)^T) and linear_w8a8 (x quantized per
   1x128 K-group, then the FP8 GEMM).
 `value` = FLOPs of the step's two linears (2 * 2MNK) / device time of the
-step, summed over ranks / max over ranks. Per-call times, TFLOP/s, weight
-GB/s and roofline fractions are reported beside it. L2 is flushed between
+whole step, summed over ranks / max over ranks; the step's time includes the
+converter and the dequantizer, so `value` is no single call's throughput --
+the per-call times, TFLOP/s, weight GB/s and roofline fractions in `calls`
+carry that. `targets` times the two linears alone on the large-token and the
+small-token (weight-streaming) shapes, each call with a clean L2, and gives
+their fractions of the measured and of the datasheet peaks with the clocks
+seen meanwhile. L2 is flushed between
 steps outside the step's CUDA events: a 512 MiB memset, then a 256 MiB read,
 so the step starts with no input in L2 and no dirty flush lines to write back.
 
@@ -37,6 +42,8 @@ if ROOT not in sys.path:
 METRIC = "block-FP8 linear TFLOP/s and weight-stream GB/s (M=512,K=5120,N=25600)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
+# B200 datasheet figures (dense): HBM3e bandwidth, BF16 and FP8 tensor throughput
+DATASHEET = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0, "fp8_tflops": 4500.0}
 FLUSH_BYTES = 512 << 20
 FLUSH_READ_BYTES = 256 << 20
 
@@ -59,6 +66,13 @@ def parse():
     ap.add_argument("--stack-mode", type=int, default=0, choices=[0, 1], help="0 W8A16, 1 W8A8")
     ap.add_argument("--stack-m", type=int, default=512)
     ap.add_argument("--stack-slots", type=int, default=2)
+    ap.add_argument("--call", default="", choices=["", "w8a16", "w8a8", "quantize_weight",
+                                                   "dequantize"],
+                    help="instead of the step: time one call on --shape (used for profiling)")
+    ap.add_argument("--shape", default="512,5120,25600", help="M,K,N for --call")
+    ap.add_argument("--reps", type=int, default=10, help="timed calls for --call")
+    ap.add_argument("--no-targets", action="store_true",
+                    help="skip the per-call timings of the large- and small-token linears")
     ap.add_argument("--no-ab", action="store_true",
                     help="skip the A/B timings of the library BF16 route and shared act quantization")
     return ap.parse_args()
@@ -237,6 +251,106 @@ def traffic_for(kernel_file: str, key: str):
     except (OSError, ValueError):
         pass
     return None
+
+
+def measure_targets(fb, dev, peaks, flush_l2, clock_sampler):
+    """Per-call device times of the two linears on the large-token shapes
+    (M = 4096, 16384; K = 5120, N = 25600: tensor-bound) and on the
+    weight-streaming sweep (M = 1, 16, 64 on the decoder's QKV, o_proj,
+    gate_up and down shapes: HBM-bound), each call alone with L2 flushed
+    before it (median over repetitions, CUDA events on the launching stream).
+    Fractions are given against the measured peaks (copy bandwidth, cuBLAS
+    BF16; FP8 = 2 x BF16) and against the datasheet figures."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(123)
+
+    def weights(N, K):
+        ldw = -(-K // 8) * 8
+        w = (torch.randn(N, ldw, device=dev, generator=g) * 0.02).to(torch.bfloat16)[:, :K]
+        q, s = fb.quantize_weight(w)
+        del w
+        return q, s
+
+    def activations(M, K):
+        x = torch.randn(M, K, device=dev, generator=g)
+        ch = torch.randperm(K, device=dev, generator=g)[:max(1, K // 100)]
+        x[:, ch] *= 20.0
+        return x.to(torch.bfloat16)
+
+    def timed(fn, reps):
+        fn()
+        ts = []
+        for _ in range(reps):
+            flush_l2()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(); fn(); b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return 1e3 * statistics.median(a.elapsed_time(b) for a, b in ts)
+
+    out = {"large_m": [], "small_m": []}
+    clock_sampler.start()
+    time.sleep(0.15)
+    K, N = 5120, 25600
+    q, s = weights(N, K)
+    for M in (4096, 16384):
+        x = activations(M, K)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws8 = torch.empty(max(1, fb.workspace_size(1, M, N, K)), dtype=torch.uint8, device=dev)
+        reps = 10 if M <= 4096 else 5
+        fl = 2.0 * M * N * K
+        for mode in ("w8a8", "w8a16"):
+            if mode == "w8a8":
+                us = timed(lambda: fb.linear_w8a8(x, q, s, out=y, workspace=ws8), reps)
+                pk, ds = FP8_OVER_BF16 * peaks["bf16_tflops"], DATASHEET["fp8_tflops"]
+            else:
+                us = timed(lambda: fb.linear_w8a16(x, q, s, out=y), reps)
+                pk, ds = peaks["bf16_tflops"], DATASHEET["bf16_tflops"]
+            tf = fl / (us * 1e-6) / 1e12
+            out["large_m"].append({"mode": mode, "M": M, "K": K, "N": N, "us": us, "tflops": tf,
+                                   "frac_measured": tf / pk, "frac_datasheet": tf / ds,
+                                   "peak_measured": pk, "peak_datasheet": ds})
+        del x, y, ws8
+    del q, s
+    shapes = [("qkv", 5120, 10240), ("o_proj", 8192, 5120), ("gate_up", 5120, 51200),
+              ("down", 25600, 5120)]
+    for name, K, N in shapes:
+        q, s = weights(N, K)
+        wbytes = N * K + 4 * s.numel()
+        for M in (1, 16, 64):
+            x = activations(M, K)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws16 = torch.empty(max(1, fb.workspace_size(0, M, N, K)), dtype=torch.uint8, device=dev)
+            ws8 = torch.empty(max(1, fb.workspace_size(1, M, N, K)), dtype=torch.uint8, device=dev)
+            for mode in ("w8a16", "w8a8"):
+                if mode == "w8a16":
+                    us = timed(lambda: fb.linear_w8a16(x, q, s, out=y, workspace=ws16), 20)
+                else:
+                    us = timed(lambda: fb.linear_w8a8(x, q, s, out=y, workspace=ws8), 20)
+                gbs = wbytes / (us * 1e-6) / 1e9
+                out["small_m"].append({"mode": mode, "layer": name, "M": M, "K": K, "N": N,
+                                       "us": us, "weight_gbs": gbs,
+                                       "frac_measured": gbs / peaks["hbm_gbs"],
+                                       "frac_datasheet": gbs / DATASHEET["hbm_gbs"]})
+            del x, y, ws16, ws8
+        del q, s
+    out["clocks"] = clock_sampler.stop()
+    torch.cuda.synchronize()
+    assert fb.read_device_error() == 0
+    w8a8_large = [r for r in out["large_m"] if r["mode"] == "w8a8"]
+    w8a16_small = [r for r in out["small_m"] if r["mode"] == "w8a16"]
+    out["north_star"] = {
+        "w8a8_m_ge_4096_min_frac_measured": min(r["frac_measured"] for r in w8a8_large),
+        "w8a8_m_ge_4096_min_frac_datasheet": min(r["frac_datasheet"] for r in w8a8_large),
+        "w8a8_target": 0.60,
+        "w8a16_m_le_64_min_frac_measured": min(r["frac_measured"] for r in w8a16_small),
+        "w8a16_m_le_64_min_frac_datasheet": min(r["frac_datasheet"] for r in w8a16_small),
+        "w8a16_target": 0.70,
+    }
+    out["timing"] = ("median of 10 (M=4096), 5 (M=16384) or 20 (small M) calls, each alone "
+                     "with L2 flushed before it; synthetic seeded weights (N(0, 0.02^2) BF16, "
+                     "converted by the library) and activations (N(0,1), 1% of channels x20)")
+    return out
 
 
 # Linears of one decoder layer of the 32B class the pages' encoder belongs to
@@ -426,6 +540,49 @@ def decode_arm(args):
     print(json.dumps(line), flush=True)
 
 
+def call_arm(args):
+    """One call on one shape, repeated: `--reps` timed calls after one
+    untimed one, L2 flushed before each, CUDA events on the launching stream.
+    Prints the median time and the call's throughput."""
+    import torch
+    import block_scaled_fp8_fp8blk_b200 as fb
+    M, K, N = (int(v) for v in args.shape.split(","))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(7)
+    ldw = -(-K // 8) * 8
+    w = (torch.randn(N, ldw, device=dev, generator=g) * 0.02).to(torch.bfloat16)[:, :K]
+    q, s = fb.quantize_weight(w)
+    x = torch.randn(M, ldw, device=dev, generator=g).to(torch.bfloat16)[:, :K]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    wd = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    mode = 0 if args.call == "w8a16" else 1
+    ws = torch.empty(max(1, fb.workspace_size(mode, M, N, K)), dtype=torch.uint8, device=dev)
+    run = {"w8a16": lambda: fb.linear_w8a16(x, q, s, out=y, workspace=ws),
+           "w8a8": lambda: fb.linear_w8a8(x, q, s, out=y, workspace=ws),
+           "quantize_weight": lambda: fb.quantize_weight(w, q=q, scale_inv=s),
+           "dequantize": lambda: fb.dequantize(q, s, out=wd)}[args.call]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.float32, device=dev)
+    run()
+    ts = []
+    for _ in range(args.reps):
+        flush.zero_()
+        flush_rd.sum()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(); run(); b.record()
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    assert fb.read_device_error() == 0
+    us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in ts)
+    NB, KB = -(-N // 128), -(-K // 128)
+    line = {"call": args.call, "M": M, "K": K, "N": N, "reps": args.reps, "us": us,
+            "weight_gbs": (N * K + 4 * NB * KB) / (us * 1e-6) / 1e9}
+    if args.call in ("w8a16", "w8a8"):
+        line["tflops"] = 2.0 * M * N * K / (us * 1e-6) / 1e12
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     from block_scaled_fp8_fp8blk_b200 import workloads
@@ -437,6 +594,10 @@ def main():
     if args.decode > 0:
         if int(os.environ.get("RANK", "0")) == 0:
             decode_arm(args)
+        return
+    if args.call:
+        if int(os.environ.get("RANK", "0")) == 0:
+            call_arm(args)
         return
     if args.impl == "reference":
         return reference_arm(args, wl)
@@ -642,6 +803,10 @@ def main():
     else:
         line["e2e"] = None
 
+    if not args.no_targets and world == 1:
+        line["targets"] = measure_targets(fb, dev, peaks, flush_l2, ClockSampler(
+            visible.split(",")[local] if visible else str(local)))
+
     # A/B, outside the step: (1) the route of FP8-less tensor cores, our
     # dequantize then a library BF16 GEMM on the expanded weight, against the
     # fused W8A16 call; (2) one activation quantization shared by sibling
@@ -658,6 +823,9 @@ def main():
             torch.cuda.synchronize()
             return 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ts)
 
+        # the route's matmul accumulates in FP32 throughout (no reduced-precision
+        # split reduction), as the parity test of this route checks it
+        torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction = False
         y_lib = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         qx, sx = fb.quantize_act(x)
         for _ in range(3):
