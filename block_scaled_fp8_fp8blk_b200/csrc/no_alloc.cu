@@ -12,7 +12,8 @@
 // The array is FP8BLK_NOALLOC_SCRATCH_BYTES (16 MiB) on every GPU that loads
 // the library, held until the process exits. Its address is looked up once
 // per device with cudaGetSymbolAddress, on the first call made while that
-// device is current.
+// device is current; that first call must not be made during stream capture
+// (it is refused with FP8BLK_ERR_INVALID_ARG).
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -34,13 +35,18 @@ std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device (host code may
-// not use the symbol itself: on the host it is only a stand-in).
-fp8blk_status scratch_address(void** out) {
+// not use the symbol itself: on the host it is only a stand-in). The lookup
+// is made once per device; a first call while `stream` is being captured is
+// refused (INVALID_ARG), since the lookup may load the module.
+fp8blk_status scratch_address(cudaStream_t stream, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FP8BLK_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return FP8BLK_ERR_UNSUPPORTED_DEVICE;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (!g_scratch_ptr[dev]) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return FP8BLK_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return FP8BLK_ERR_INVALID_ARG;
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FP8BLK_ERR_CUDA;
     g_scratch_ptr[dev] = p;
@@ -48,8 +54,6 @@ fp8blk_status scratch_address(void** out) {
   *out = g_scratch_ptr[dev];
   return FP8BLK_OK;
 }
-
-bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 }  // namespace
 }  // namespace fp8blk
@@ -60,33 +64,23 @@ extern "C" fp8blk_status fp8blk_linear_w8a8_noalloc(const void* x, int64_t ldx, 
                                                     int64_t ldq, const float* scale_inv, void* y,
                                                     int64_t ldy, int64_t M, int64_t N, int64_t K,
                                                     fp8blk_stream stream) {
-  if (M < 0 || N < 0 || K < 0) return FP8BLK_ERR_INVALID_ARG;
+  // The checks of fp8blk_linear_w8a8, without its workspace.
+  fp8blk_status st = validate_linear(x, ldx, q, ldq, scale_inv, y, ldy, M, N, K, nullptr, 0, 0);
+  if (st != FP8BLK_OK) return st;
   if (M == 0 || N == 0) return FP8BLK_OK;
-  if (!y || ldy < N) return FP8BLK_ERR_INVALID_ARG;
-  if (ldy % 8 || !is_aligned(y, 16)) return FP8BLK_ERR_ALIGNMENT;
-  if (K == 0) {
-    // An empty sum: y = 0 (no scratch involved).
-    Launch L;
-    fp8blk_status st = current_launch(stream, &L);
-    if (st != FP8BLK_OK) return st;
+  Launch L;
+  st = current_launch(stream, &L);
+  if (st != FP8BLK_OK) return st;
+  if (K == 0)  // an empty sum: y = 0 (no scratch involved)
     return cudaMemset2DAsync(y, static_cast<size_t>(ldy) * 2, 0, static_cast<size_t>(N) * 2,
                              static_cast<size_t>(M), L.stream) == cudaSuccess
                ? FP8BLK_OK
                : FP8BLK_ERR_CUDA;
-  }
-  if (!x || !q || !scale_inv || ldx < K || ldq < K) return FP8BLK_ERR_INVALID_ARG;
-  if (M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL || K > 0x7FFFFFFFLL) return FP8BLK_ERR_INVALID_ARG;
-  if (ldx % 8 || ldq % 16 || !is_aligned(x, 16) || !is_aligned(q, 16) || !is_aligned(scale_inv, 4))
-    return FP8BLK_ERR_ALIGNMENT;
   // Same layout as the W8A8 workspace; refuse problems that do not fit.
   const size_t need = fp8blk_workspace_size(1, M, N, K);
   if (need > static_cast<size_t>(FP8BLK_NOALLOC_SCRATCH_BYTES)) return FP8BLK_ERR_WORKSPACE;
-
-  Launch L;
-  fp8blk_status st = current_launch(stream, &L);
-  if (st != FP8BLK_OK) return st;
   void* scratch = nullptr;
-  st = scratch_address(&scratch);
+  st = scratch_address(L.stream, &scratch);
   if (st != FP8BLK_OK) return st;
 
   uint8_t* qx = static_cast<uint8_t*>(scratch);

@@ -170,7 +170,7 @@ FP8BLK_EXPORT fp8blk_status fp8blk_linear_w8a8(const void* x, int64_t ldx, const
  *    FP8BLK_ERR_WORKSPACE before anything is launched.
  *  - The first call on a device (with that device current) looks up the
  *    array's device address once; make that first call before any stream
- *    capture.
+ *    capture (a first call on a capturing stream returns INVALID_ARG).
  *  - All calls share the one array: calls that can overlap on the GPU (on
  *    different streams, or from different threads) race on it and must be
  *    ordered by the caller.
