@@ -260,6 +260,30 @@ def test_w8a16_one_hot_rows_reproduce_dequantized_weight():
         assert np.array_equal(got[i], deq[:, k])
 
 
+@pytest.mark.parametrize("M", [16, 128, 300])
+def test_w8a16_every_code_through_the_gemm(M):
+    """Every E4M3 code (NaNs excepted) as a weight, identity activations: each
+    output is one code times its block scale, rounded once, so y must equal
+    the dequantized weight bit for bit (zeros as +0) -- this pins the
+    kernel's FP8 -> BF16 expansion on all 254 finite codes, subnormals
+    included, on the small-token (M <= 128) and the two-sub-tile (M > 128)
+    paths."""
+    N, K = 256, 128
+    q = (np.arange(N * K, dtype=np.int64).reshape(N, K) % 256).astype(np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x00
+    s = np.array([[1.0], [2.0 ** -100]], dtype=np.float32)
+    x = np.zeros((M, K), np.float32)
+    x[np.arange(M), np.arange(M) % K] = 1.0
+    y = fb.linear_w8a16(to_dev_bf16(synth.bf16_bits(synth.to_bf16(x))), to_dev_u8(q),
+                        torch.from_numpy(s).to(DEV))
+    got = bf16_bits(y)
+    want = oracle.dequantize(q, s)[:, np.arange(M) % K].T.copy()   # [M, N]
+    # a zero code's product is summed with the other columns' zero products,
+    # so it comes out +0 whatever its sign (IEEE: -0 + +0 = +0)
+    want[want == 0x8000] = 0
+    assert np.array_equal(got, want)
+
+
 def test_repeat_calls_are_deterministic():
     wl = W.Workload("m300_k640_n512", 300, 640, 512)
     wb, q, s = weight_case(wl)
