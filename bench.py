@@ -44,6 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP8_OVER_BF16 = 2.0   # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
 # B200 datasheet figures (dense): HBM3e bandwidth, BF16 and FP8 tensor throughput
 DATASHEET = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0, "fp8_tflops": 4500.0}
+ROTATE_BYTES = 2 * 126 * 10**6   # back-to-back timings rotate weights over twice the L2
 FLUSH_BYTES = 512 << 20
 FLUSH_READ_BYTES = 256 << 20
 
@@ -134,7 +135,8 @@ class ClockSampler:
         reasons = sorted({names[i] for r in loaded for i in range(1, 5) if r[3][i] == "Active"})
         return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": rows[0][1],
                 "reasons": reasons, "samples": len(loaded),
-                "power_w_max": max(r[2] for r in rows)}
+                "sm_mhz_all_samples": statistics.median(r[0] for r in rows),
+                "samples_all": len(rows), "power_w_max": max(r[2] for r in rows)}
 
 
 # --------------------------------------------------------------- oracle arm
@@ -288,7 +290,75 @@ def measure_targets(fb, dev, peaks, flush_l2, clock_sampler):
         torch.cuda.synchronize()
         return 1e3 * statistics.median(a.elapsed_time(b) for a, b in ts)
 
+    def back_to_back(call, copies, rounds=4):
+        """Per-call time of calls run back to back from a CUDA graph, each on
+        the next weight copy in turn (a pass over the copies is twice the L2,
+        so every call streams its weight from HBM): the decode-time regime,
+        where one linear follows another and launch latency overlaps the
+        kernel before."""
+        cs = torch.cuda.Stream()
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cs):
+            for qq, ss in copies:
+                call(qq, ss)
+        torch.cuda.current_stream().wait_stream(cs)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cs):
+            for _ in range(rounds):
+                for qq, ss in copies:
+                    call(qq, ss)
+        graph.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(3):
+            flush_l2()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(); graph.replay(); b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        del graph
+        return 1e3 * statistics.median(a.elapsed_time(b) for a, b in ts) / (rounds * len(copies))
+
     out = {"large_m": [], "small_m": []}
+    # The weight-streaming sweep runs first, after a short idle: the
+    # tensor-bound calls below draw enough power to lower the clocks for a
+    # while, which short latency-bound calls would feel.
+    torch.cuda.synchronize()
+    time.sleep(1.0)
+    clock_sampler.start()
+    time.sleep(0.15)
+    shapes = [("qkv", 5120, 10240), ("o_proj", 8192, 5120), ("gate_up", 5120, 51200),
+              ("down", 25600, 5120)]
+    for name, K, N in shapes:
+        # enough copies of the weight that one pass over them is twice the L2
+        copies = [weights(N, K)]
+        wbytes = N * K + 4 * copies[0][1].numel()
+        while len(copies) < max(2, -(-ROTATE_BYTES // wbytes)):
+            copies.append(weights(N, K))
+        q, s = copies[0]
+        for M in (1, 16, 64):
+            x = activations(M, K)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws16 = torch.empty(max(1, fb.workspace_size(0, M, N, K)), dtype=torch.uint8, device=dev)
+            ws8 = torch.empty(max(1, fb.workspace_size(1, M, N, K)), dtype=torch.uint8, device=dev)
+            for mode in ("w8a16", "w8a8"):
+                f = fb.linear_w8a16 if mode == "w8a16" else fb.linear_w8a8
+                ws = ws16 if mode == "w8a16" else ws8
+                us = timed(lambda: f(x, q, s, out=y, workspace=ws), 20)
+                us_b2b = back_to_back(lambda qq, ss: f(x, qq, ss, out=y, workspace=ws), copies)
+                gbs, gbs_b2b = wbytes / (us * 1e-6) / 1e9, wbytes / (us_b2b * 1e-6) / 1e9
+                out["small_m"].append({"mode": mode, "layer": name, "M": M, "K": K, "N": N,
+                                       "us": us, "weight_gbs": gbs,
+                                       "frac_measured": gbs / peaks["hbm_gbs"],
+                                       "frac_datasheet": gbs / DATASHEET["hbm_gbs"],
+                                       "us_back_to_back": us_b2b, "weight_gbs_back_to_back": gbs_b2b,
+                                       "frac_measured_back_to_back": gbs_b2b / peaks["hbm_gbs"],
+                                       "frac_datasheet_back_to_back": gbs_b2b / DATASHEET["hbm_gbs"],
+                                       "weight_copies": len(copies)})
+            del x, y, ws16, ws8
+        del q, s, copies
+    out["clocks_small_m"] = clock_sampler.stop()
     clock_sampler.start()
     time.sleep(0.15)
     K, N = 5120, 25600
@@ -312,34 +382,14 @@ def measure_targets(fb, dev, peaks, flush_l2, clock_sampler):
                                    "peak_measured": pk, "peak_datasheet": ds})
         del x, y, ws8
     del q, s
-    shapes = [("qkv", 5120, 10240), ("o_proj", 8192, 5120), ("gate_up", 5120, 51200),
-              ("down", 25600, 5120)]
-    for name, K, N in shapes:
-        q, s = weights(N, K)
-        wbytes = N * K + 4 * s.numel()
-        for M in (1, 16, 64):
-            x = activations(M, K)
-            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-            ws16 = torch.empty(max(1, fb.workspace_size(0, M, N, K)), dtype=torch.uint8, device=dev)
-            ws8 = torch.empty(max(1, fb.workspace_size(1, M, N, K)), dtype=torch.uint8, device=dev)
-            for mode in ("w8a16", "w8a8"):
-                if mode == "w8a16":
-                    us = timed(lambda: fb.linear_w8a16(x, q, s, out=y, workspace=ws16), 20)
-                else:
-                    us = timed(lambda: fb.linear_w8a8(x, q, s, out=y, workspace=ws8), 20)
-                gbs = wbytes / (us * 1e-6) / 1e9
-                out["small_m"].append({"mode": mode, "layer": name, "M": M, "K": K, "N": N,
-                                       "us": us, "weight_gbs": gbs,
-                                       "frac_measured": gbs / peaks["hbm_gbs"],
-                                       "frac_datasheet": gbs / DATASHEET["hbm_gbs"]})
-            del x, y, ws16, ws8
-        del q, s
-    out["clocks"] = clock_sampler.stop()
+    out["clocks_large_m"] = clock_sampler.stop()
     torch.cuda.synchronize()
     assert fb.read_device_error() == 0
     w8a8_large = [r for r in out["large_m"] if r["mode"] == "w8a8"]
     w8a16_small = [r for r in out["small_m"] if r["mode"] == "w8a16"]
     out["north_star"] = {
+        "w8a16_m_le_64_min_frac_measured_back_to_back": min(r["frac_measured_back_to_back"]
+                                                            for r in w8a16_small),
         "w8a8_m_ge_4096_min_frac_measured": min(r["frac_measured"] for r in w8a8_large),
         "w8a8_m_ge_4096_min_frac_datasheet": min(r["frac_datasheet"] for r in w8a8_large),
         "w8a8_target": 0.60,
@@ -347,9 +397,11 @@ def measure_targets(fb, dev, peaks, flush_l2, clock_sampler):
         "w8a16_m_le_64_min_frac_datasheet": min(r["frac_datasheet"] for r in w8a16_small),
         "w8a16_target": 0.70,
     }
-    out["timing"] = ("median of 10 (M=4096), 5 (M=16384) or 20 (small M) calls, each alone "
-                     "with L2 flushed before it; synthetic seeded weights (N(0, 0.02^2) BF16, "
-                     "converted by the library) and activations (N(0,1), 1% of channels x20)")
+    out["timing"] = ("per call: median of 10 (M=4096), 5 (M=16384) or 20 (small M) calls, "
+                     "each alone with L2 flushed before it; back to back (small M): a CUDA "
+                     "graph of 4 rounds over weight copies totalling twice the L2, per call; "
+                     "synthetic seeded weights (N(0, 0.02^2) BF16, converted by the library) "
+                     "and activations (N(0,1), 1% of channels x20)")
     return out
 
 
