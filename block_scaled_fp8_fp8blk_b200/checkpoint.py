@@ -166,11 +166,19 @@ def save_checkpoint(out_dir: str, tensors: dict, config: dict | None = None,
                                    metadata={"format": "pt"})
         for n in names:
             weight_map[n] = fname
+    return _write_index_and_config(out_dir, weight_map, total, config,
+                                   any(t.dtype == torch.float8_e4m3fn for t in tensors.values()))
+
+
+def _write_index_and_config(out_dir: str, weight_map: dict, total: int, config: dict | None,
+                            has_fp8: bool) -> dict:
+    """The index (tensor -> shard, total bytes) and config.json, with
+    quantization_config when the checkpoint holds E4M3 weights."""
     index = {"metadata": {"total_size": total}, "weight_map": dict(sorted(weight_map.items()))}
     with open(os.path.join(out_dir, INDEX_NAME), "w") as f:
         json.dump(index, f, indent=2)
     cfg = dict(config or {})
-    if any(t.dtype == torch.float8_e4m3fn for t in tensors.values()):
+    if has_fp8:
         cfg["quantization_config"] = dict(QUANTIZATION_CONFIG)
     with open(os.path.join(out_dir, "config.json"), "w") as f:
         json.dump(cfg, f, indent=2)
@@ -205,18 +213,52 @@ def load_checkpoint(in_dir: str, names: Iterable[str] | None = None) -> tuple[di
 def convert_checkpoint(src_dir: str, dst_dir: str, is_linear: Callable = default_is_linear,
                        max_shard_bytes: int = 5 * 10**9) -> dict:
     """BF16 checkpoint (index + shards, or a single ``model.safetensors``) ->
-    block-FP8 checkpoint, converting one source shard at a time on the GPU."""
+    block-FP8 checkpoint. Source shards are converted one at a time on the
+    GPU and output shards are written as they fill, so the host holds at most
+    one source shard, its converted tensors and one output shard (each output
+    shard up to ``max_shard_bytes`` unless one tensor is bigger). Shards are
+    written under temporary names and renamed model-XXXXX-of-YYYYY once their
+    count is known; returns the index."""
     idx_path = os.path.join(src_dir, INDEX_NAME)
     if os.path.exists(idx_path):
         with open(idx_path) as f:
             files = sorted(set(json.load(f)["weight_map"].values()))
     else:
         files = ["model.safetensors"]
-    converted = {}
+    os.makedirs(dst_dir, exist_ok=True)
+    parts: list = []          # (temporary file name, tensor names)
+    pending: dict = {}
+    state = {"bytes": 0, "total": 0, "fp8": False}
+
+    def write_part():
+        tmp = f"model-part-{len(parts):05d}.safetensors"
+        state["total"] += write_safetensors(os.path.join(dst_dir, tmp), pending,
+                                            metadata={"format": "pt"})
+        parts.append((tmp, sorted(pending)))
+        pending.clear()
+        state["bytes"] = 0
+
     for fname in files:
-        converted.update(quantize_state_dict(read_safetensors(os.path.join(src_dir, fname)),
-                                             is_linear))
-    return save_checkpoint(dst_dir, converted, _read_config(src_dir), max_shard_bytes)
+        converted = quantize_state_dict(read_safetensors(os.path.join(src_dir, fname)), is_linear)
+        for name in sorted(converted):
+            t = converted[name]
+            nb = t.numel() * t.element_size()
+            if pending and state["bytes"] + nb > max_shard_bytes:
+                write_part()
+            pending[name] = t
+            state["bytes"] += nb
+            state["fp8"] = state["fp8"] or t.dtype == torch.float8_e4m3fn
+        del converted
+    if pending or not parts:
+        write_part()
+    weight_map = {}
+    for i, (tmp, names) in enumerate(parts):
+        final = f"model-{i + 1:05d}-of-{len(parts):05d}.safetensors"
+        os.replace(os.path.join(dst_dir, tmp), os.path.join(dst_dir, final))
+        for n in names:
+            weight_map[n] = final
+    return _write_index_and_config(dst_dir, weight_map, state["total"], _read_config(src_dir),
+                                   state["fp8"])
 
 
 def linear_weights(tensors: dict, name: str, device: str | torch.device = "cuda",

@@ -147,3 +147,33 @@ def test_convert_checkpoint_without_linears_passes_through(tmp_path, monkeypatch
         same(back[k], v)
     with pytest.raises(RuntimeError, match="CUDA"):           # a linear still needs the GPU
         ck.convert_checkpoint(src, str(tmp_path / "dst2"))
+
+
+def test_convert_checkpoint_writes_shards_as_they_fill(tmp_path, monkeypatch):
+    """Output shards are written while converting, each up to the size limit
+    (one tensor larger than the limit gets a shard of its own), renamed
+    model-XXXXX-of-YYYYY at the end with no temporary file left behind; the
+    index covers every tensor once."""
+    monkeypatch.setattr(torch.cuda, "is_available", lambda: False)
+    g = torch.Generator().manual_seed(10)
+    src_t = {f"model.layers.{i}.norm.weight": torch.randn(16 * (i + 1), generator=g).to(torch.bfloat16)
+             for i in range(7)}
+    src_t["model.embed_tokens.weight"] = torch.randn(30, 20, generator=g).to(torch.bfloat16)  # 1200 B
+    src = str(tmp_path / "src")
+    ck.save_checkpoint(src, src_t, {"model_type": "toy"}, max_shard_bytes=100)
+    dst = str(tmp_path / "dst")
+    limit = 300
+    idx = ck.convert_checkpoint(src, dst, is_linear=lambda n, t: False, max_shard_bytes=limit)
+    files = sorted(set(idx["weight_map"].values()))
+    assert len(files) >= 3
+    assert files == [f"model-{i + 1:05d}-of-{len(files):05d}.safetensors" for i in range(len(files))]
+    assert sorted(os.listdir(dst)) == sorted(files + [ck.INDEX_NAME, "config.json"])
+    assert set(idx["weight_map"]) == set(src_t)
+    for f in files:
+        names = [n for n, v in idx["weight_map"].items() if v == f]
+        nbytes = sum(src_t[n].numel() * 2 for n in names)
+        assert nbytes <= limit or len(names) == 1
+    assert idx["metadata"]["total_size"] == sum(t.numel() * 2 for t in src_t.values())
+    back, _ = ck.load_checkpoint(dst)
+    for k, v in src_t.items():
+        same(back[k], v)
