@@ -162,6 +162,14 @@ fp8blk_status validate_linear(const void* x, int64_t ldx, const uint8_t* q, int6
   return FP8BLK_OK;
 }
 
+// The workspace a linear call cannot run without (fp8blk_workspace_size
+// gives the size that enables every path; for W8A16 above 128 tokens the
+// stream-K tail it enables is optional).
+size_t required_workspace(int mode, int64_t M, int64_t N, int64_t K) {
+  if (mode == 0) return (M <= 0 || N <= 0 || K <= 0) ? 0 : w8a16_workspace_required(M, N, K);
+  return fp8blk_workspace_size(mode, M, N, K);
+}
+
 // The launch context of the current device (stream, error word, SM count),
 // for entry points defined in other files.
 fp8blk_status current_launch(fp8blk_stream stream, Launch* L) { return make_launch(stream, L); }
@@ -251,7 +259,7 @@ fp8blk_status fp8blk_linear_w8a16(const void* x, int64_t ldx, const uint8_t* q, 
   Launch L;
   bool done = false;
   fp8blk_status st = check_linear(x, ldx, q, ldq, scale_inv, y, ldy, M, N, K, workspace,
-                                  workspace_bytes, fp8blk_workspace_size(0, M, N, K), stream, &L,
+                                  workspace_bytes, required_workspace(0, M, N, K), stream, &L,
                                   &done);
   if (st != FP8BLK_OK || done) return st;
   return cuda_status(launch_w8a16_gemm(L, static_cast<const uint16_t*>(x), ldx, q, ldq, scale_inv,
@@ -290,7 +298,7 @@ fp8blk_status fp8blk_linear_sequence(const fp8blk_linear_args* jobs, int64_t njo
     if (j.mode != 0 && j.mode != 1) return FP8BLK_ERR_INVALID_ARG;
     const fp8blk_status st = validate_linear(j.x, j.ldx, j.q, j.ldq, j.scale_inv, j.y, j.ldy, j.M,
                                              j.N, j.K, workspace, workspace_bytes,
-                                             fp8blk_workspace_size(j.mode, j.M, j.N, j.K));
+                                             required_workspace(j.mode, j.M, j.N, j.K));
     if (st != FP8BLK_OK) return st;
   }
   Launch L;

@@ -123,40 +123,42 @@ __device__ __forceinline__ uint32_t ring_parity(int item, int depth) {
   return static_cast<uint32_t>((item / depth) & 1);
 }
 
-// The slabs one CTA runs, as a run of segments (tile, [kb0, kb1)): whole
-// tiles blockIdx.x, + gridDim.x, ... (round robin), or with stream-K the
-// contiguous range [c U / G, (c + 1) U / G) of the U = tiles x KB slabs in
-// tile-major order (c = blockIdx.x, G = gridDim.x), which gives every CTA the
-// same number of slabs within one. Under stream-K a tile may be split across
-// consecutive CTAs; only a CTA's first and last segments can be partial.
+// The slabs one CTA runs, as a run of segments (tile, [kb0, kb1)). Tiles
+// [0, dp_tiles) run whole, round robin (CTA c takes c, c + G, ...; G =
+// gridDim.x); the U = (tiles - dp_tiles) x KB slabs of the other tiles, in
+// tile-major order, run stream-K: CTA c takes the contiguous range
+// [c U / G, (c + 1) U / G), so every CTA gets the same share within one slab.
+// A stream-K tile may be split across consecutive CTAs; only a CTA's first
+// and last stream-K segments can be partial. dp_tiles = 0 is pure stream-K,
+// dp_tiles = tiles pure round robin.
+// (Slab counts fit in 32 bits: the host checks tiles x KB.)
 struct Schedule {
-  int64_t u, end, first;
-  int tile, KB, ntiles;
-  bool streamk;
-  __device__ Schedule(bool sk, int kb_per_tile, int tiles)
-      : tile(static_cast<int>(blockIdx.x)), KB(kb_per_tile), ntiles(tiles), streamk(sk) {
-    const int64_t U = static_cast<int64_t>(tiles) * kb_per_tile;
-    first = u = U * blockIdx.x / gridDim.x;
-    end = U * (blockIdx.x + 1) / gridDim.x;
+  int u, end, first;
+  int tile, KB, dp_tiles;
+  __device__ Schedule(int kb_per_tile, int tiles, int dp)
+      : tile(static_cast<int>(blockIdx.x)), KB(kb_per_tile), dp_tiles(dp) {
+    const int64_t U = static_cast<int64_t>(tiles - dp) * kb_per_tile;
+    first = u = static_cast<int>(U * blockIdx.x / gridDim.x);
+    end = static_cast<int>(U * (blockIdx.x + 1) / gridDim.x);
   }
   __device__ int slabs() const {
-    if (streamk) return static_cast<int>(end - first);
-    return tile < ntiles ? ((ntiles - 1 - tile) / static_cast<int>(gridDim.x) + 1) * KB : 0;
+    const int dp = tile < dp_tiles ? ((dp_tiles - 1 - tile) / static_cast<int>(gridDim.x) + 1) * KB : 0;
+    return dp + (end - first);
   }
   __device__ bool next(int& t, int& kb0, int& kb1) {
-    if (streamk) {
-      if (u >= end) return false;
-      t = static_cast<int>(u / KB);
-      kb0 = static_cast<int>(u - static_cast<int64_t>(t) * KB);
-      kb1 = static_cast<int>(min(static_cast<int64_t>(KB), kb0 + (end - u)));
-      u += kb1 - kb0;
+    if (tile < dp_tiles) {
+      t = tile;
+      kb0 = 0;
+      kb1 = KB;
+      tile += static_cast<int>(gridDim.x);
       return true;
     }
-    if (tile >= ntiles) return false;
-    t = tile;
-    kb0 = 0;
-    kb1 = KB;
-    tile += static_cast<int>(gridDim.x);
+    if (u >= end) return false;
+    const int lt = u / KB;
+    t = dp_tiles + lt;
+    kb0 = u - lt * KB;
+    kb1 = min(KB, kb0 + (end - u));
+    u += kb1 - kb0;
     return true;
   }
 };
@@ -221,7 +223,7 @@ template <int BT, int NSUB>
 __global__ void __launch_bounds__(512, 1)
     w8a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_x,
                       const float* __restrict__ sw, __nv_bfloat16* __restrict__ y, int64_t ldy,
-                      int M, int N, int KB, int mtiles, int ntiles_total, int streamk,
+                      int M, int N, int KB, int mtiles, int ntiles_total, int dp_tiles,
                       int early_weights, float* __restrict__ part, unsigned* __restrict__ err) {
   using C = W8A16Cfg<BT, NSUB>;
   extern __shared__ uint8_t smem_raw[];
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(512, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + C::PB * 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total_slabs = Schedule(streamk != 0, KB, ntiles_total).slabs();
+  const int total_slabs = Schedule(KB, ntiles_total, dp_tiles).slabs();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::QS; ++s) {
@@ -272,17 +274,17 @@ __global__ void __launch_bounds__(512, 1)
   pdl_launch_dependents();
 
   // Each warpgroup sets its register budget at the top of its role:
-  // 128 x (56 + 80 + 184 + 184) = 64512 of the 65536 the block holds.
+  // 128 x (64 + 72 + 184 + 184) = 64512 of the 65536 the block holds.
   const int wg = warp >> 2;
   if (wg == 0) {
-    setmaxnreg_dec<56>();
+    setmaxnreg_dec<64>();
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------ weight-code producer
       tma_prefetch_map(&tm_q);
       if (!early_weights) pdl_wait();
       int j = 0;  // slab counter (across tiles)
       bool ok = true;
-      Schedule sc(streamk != 0, KB, ntiles_total);
+      Schedule sc(KB, ntiles_total, dp_tiles);
       int tile, kb0, kb1;
       while (ok && sc.next(tile, kb0, kb1)) {
         const int n0 = (tile / mtiles) * 128;
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(512, 1)
       pdl_wait();
       int i = 0;  // item counter (across tiles)
       bool ok = true;
-      Schedule sc(streamk != 0, KB, ntiles_total);
+      Schedule sc(KB, ntiles_total, dp_tiles);
       int tile, kb0, kb1;
       while (ok && sc.next(tile, kb0, kb1)) {
         const int m0 = (tile % mtiles) * (BT * NSUB);
@@ -368,7 +370,7 @@ __global__ void __launch_bounds__(512, 1)
       if (last >= 0) mbar_wait(&done[last % C::RD], ring_parity(last, C::RD), err, kErrWaitMma);
     }
   } else if (wg == 1) {
-    setmaxnreg_dec<80>();
+    setmaxnreg_dec<72>();
     expand_slabs<C, NSUB>(0, total_slabs, sQ, tmem, qfull, qempty, afull, done, err);
   } else {
     setmaxnreg_inc<184>();
@@ -386,16 +388,19 @@ __global__ void __launch_bounds__(512, 1)
       const int rr = lane >> 1, hh = lane & 1;  // row and half this lane stores
       int j = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
+      bool first_sk = true;  // the next stream-K segment is this CTA's first
+      Schedule sc(KB, ntiles_total, dp_tiles);
+      int tile, kb0, kb1;
+      while (ok && sc.next(tile, kb0, kb1)) {
         const int m0 = (tile % mtiles) * (BT * NSUB), n0 = (tile / mtiles) * 128;
         const float* sw_row = sw + static_cast<int64_t>(n0 >> 7) * KB;
         uint64_t acc[64];  // acc[32t + p]: tokens 128t + 64h + 2p and 2p + 1
 #pragma unroll
         for (int e = 0; e < 64; ++e) acc[e] = 0ull;
-        float s_next = __ldg(sw_row);
-        for (int kb = 0; kb < KB && ok; ++kb, ++j) {
+        float s_next = __ldg(sw_row + kb0);
+        for (int kb = kb0; kb < kb1 && ok; ++kb, ++j) {
           const float s = s_next;
-          if (kb + 1 < KB) s_next = __ldg(sw_row + kb + 1);
+          if (kb + 1 < kb1) s_next = __ldg(sw_row + kb + 1);
           const uint64_t s2 = pack_f32x2(s, s);
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
@@ -420,6 +425,28 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
         if (!ok) break;
+        const int slot = first_sk ? 0 : 1;
+        if (tile >= dp_tiles) first_sk = false;
+        if (kb0 != 0 || kb1 != KB) {
+          // Part of a stream-K tile: the FP32 partial goes to slot (CTA,
+          // first or last stream-K segment) of the workspace, [256 tokens]
+          // [128 weight rows] with the weight row fastest;
+          // w8a16_streamk_fixup adds the slots.
+          float* dst = part + (static_cast<int64_t>(blockIdx.x) * 2 + slot) * (BT * NSUB * 128) +
+                       quad * 32 + lane;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+#pragma unroll
+            for (int pp = 0; pp < 32; ++pp) {
+              float lo, hi;
+              asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc[32 * t + pp]));
+              const int mloc = 128 * t + 64 * h + 2 * pp;
+              dst[mloc * 128] = lo;
+              dst[(mloc + 1) * 128] = hi;
+            }
+          }
+          continue;
+        }
         // Output: sixteen tokens at a time through shared memory as rows of
         // 32 BF16 (this warp's columns of y), then 32-byte stores per lane.
         const int nw = n0 + quad * 32;  // first column of this warp
@@ -457,7 +484,7 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::TMEM_P;
       int j = 0;
       bool ok = true;
-      Schedule sc(streamk != 0, KB, ntiles_total);
+      Schedule sc(KB, ntiles_total, dp_tiles);
       int tile, kb0, kb1;
       bool first_segment = true;
       while (ok && sc.next(tile, kb0, kb1)) {
@@ -598,33 +625,36 @@ SplitTiles split_tiles(int64_t ntiles, int64_t KB, int64_t G) {
 
 // Stream-K fix-up: y of every split tile, the sum of its contributors' FP32
 // partials in slab order, rounded once to BF16. Block (i, g) handles split
-// tile i for tokens [8 g, 8 g + 8) with one thread per weight row and token
-// parity, every partial load issued before the sums. Tiles run by a single
-// CTA were written directly. Launched as a programmatic dependent of the
-// GEMM: it waits for the GEMM grid to complete before it reads a partial.
-template <int BT>
+// tile i for tokens [8 g, 8 g + 8) of its TOK with one thread per weight row
+// and token parity, every partial load issued before the sums. Tiles run by
+// a single CTA were written directly. Launched as a programmatic dependent
+// of the GEMM: it waits for the GEMM grid to complete before it reads a
+// partial.
+template <int TOK>
 __global__ void __launch_bounds__(256) w8a16_streamk_fixup(const __grid_constant__ SplitTiles st,
                                                            const float* __restrict__ part,
                                                            uint16_t* __restrict__ y, int64_t ldy,
-                                                           int M, int N) {
+                                                           int M, int N, int mtiles) {
   pdl_launch_dependents();  // the next linear may be scheduled; it waits for this grid
   pdl_wait();
   const int i = static_cast<int>(blockIdx.x);
   const int r = threadIdx.x & 127;
-  const int n = st.tile[i] * 128 + r;
+  const int t = st.tile[i];
+  const int n = (t / mtiles) * 128 + r;
   if (n >= N) return;
+  const int m0 = (t % mtiles) * TOK;
   const int c0 = st.c0[i], nc = st.ncontrib[i], slot0 = st.slot0[i];
   const int mbase = static_cast<int>(blockIdx.y) * 8 + (threadIdx.x >> 7);
   float acc[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) acc[u] = 0.0f;
   for (int c = 0; c < nc; ++c) {
-    const float* p = part + (static_cast<int64_t>(c0 + c) * 2 + (c == 0 ? slot0 : 0)) * (BT * 128) + r;
+    const float* p = part + (static_cast<int64_t>(c0 + c) * 2 + (c == 0 ? slot0 : 0)) * (TOK * 128) + r;
     float v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int m = mbase + 2 * u;
-      v[u] = m < M && m < BT ? p[m * 128] : 0.0f;
+      v[u] = m < TOK && m0 + m < M ? p[m * 128] : 0.0f;
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) acc[u] += v[u];
@@ -632,17 +662,23 @@ __global__ void __launch_bounds__(256) w8a16_streamk_fixup(const __grid_constant
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int m = mbase + 2 * u;
-    if (m < M && m < BT)
-      y[static_cast<int64_t>(m) * ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[u]));
+    if (m < TOK && m0 + m < M)
+      y[static_cast<int64_t>(m0 + m) * ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[u]));
   }
 }
 
+// Workspace bytes of a stream-K launch with grid CTAs and TOK-token tiles:
+// two FP32 partial slots of [TOK][128] per CTA.
+size_t streamk_bytes(int64_t grid, int tok) {
+  return static_cast<size_t>(grid) * 2 * tok * 128 * sizeof(float);
+}
 
 template <int BT, int NSUB>
 cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                       int64_t ldq, const float* sw, uint16_t* y, int64_t ldy, int64_t M,
                       int64_t N, int64_t K, void* ws, size_t ws_bytes, bool early_weights) {
   using C = W8A16Cfg<BT, NSUB>;
+  constexpr int TOK = BT * NSUB;
   CUtensorMap tq, tx;
   if (!make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, N, ldq, 128, 128))
     return cudaErrorInvalidValue;
@@ -658,23 +694,42 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
       cudaFuncAttributes fa;
       cudaError_t r = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kern));
       if (r != cudaSuccess) return r;
-      return fa.numRegs * C::THREADS < 128 * (56 + 80 + 184 + 184) ? cudaErrorInvalidConfiguration
+      return fa.numRegs * C::THREADS < 128 * (64 + 72 + 184 + 184) ? cudaErrorInvalidConfiguration
                                                                    : cudaSuccess;
     }();
     if (regs != cudaSuccess) return regs;
   }
-  const int64_t mtiles = cdiv(M, BT * NSUB), tiles = mtiles * cdiv(N, 128);
+  const int64_t mtiles = cdiv(M, TOK), tiles = mtiles * cdiv(N, 128);
   // Slab and item counters are 32-bit per CTA.
   if (tiles * cdiv(K, 128) * NSUB > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  // One token tile (M <= 128): stream-K over the slabs, so every SM streams
-  // the same share of the weights however few 128-row tiles there are.
   const int64_t KB = cdiv(K, 128);
-  const bool streamk = NSUB == 1;
-  int64_t grid = streamk ? tiles * KB : tiles;
-  const int64_t cap = streamk ? (L.num_sms < kStreamKMaxCtas ? L.num_sms : kStreamKMaxCtas) : L.num_sms;
-  if (grid > cap) grid = cap;
-  if (streamk && (!ws || ws_bytes < static_cast<size_t>(grid) * 2 * BT * 128 * sizeof(float)))
-    return cudaErrorInvalidValue;
+  const int64_t G = L.num_sms < kStreamKMaxCtas ? L.num_sms : kStreamKMaxCtas;
+  int64_t dp_tiles, grid;
+  if (NSUB == 1) {
+    // One token tile (M <= 128): stream-K over all the slabs, so every SM
+    // streams the same share of the weights however few tiles there are.
+    dp_tiles = 0;
+    grid = tiles * KB < G ? tiles * KB : G;
+    if (!ws || ws_bytes < streamk_bytes(grid, TOK)) return cudaErrorInvalidValue;
+  } else {
+    // Whole tiles round robin. When the last wave of tiles would leave at
+    // least 15% of the SM time idle, and the workspace allows, the tiles of
+    // that wave run stream-K over all CTAs instead. (Below that the partial
+    // round trip and the fix-up cost what the even split saves: at 10% idle
+    // -- 400 tiles on 148 SMs -- both ran in the same time.)
+    const int64_t waves = tiles / G, rem = tiles - waves * G;
+    const int64_t tail_grid = waves > 0 ? G : (rem * KB < G ? rem * KB : G);
+    const bool tail_sk = rem > 0 && (G - rem) * 100 >= 15 * (waves + 1) * G && tail_grid >= 2 && ws &&
+                         reinterpret_cast<uintptr_t>(ws) % 256 == 0 &&
+                         ws_bytes >= streamk_bytes(tail_grid, TOK);
+    if (tail_sk) {
+      dp_tiles = waves * G;
+      grid = tail_grid;
+    } else {
+      dp_tiles = tiles;
+      grid = tiles < L.num_sms ? tiles : L.num_sms;
+    }
+  }
   // A programmatic dependent of the kernel before it in the stream (its set-up
   // overlaps that kernel's tail; see the kernel for what waits).
   {
@@ -690,14 +745,16 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, tq, tx, sw, reinterpret_cast<__nv_bfloat16*>(y), ldy,
                            static_cast<int>(M), static_cast<int>(N), static_cast<int>(KB),
-                           static_cast<int>(mtiles), static_cast<int>(tiles), streamk ? 1 : 0,
-                           early_weights ? 1 : 0, static_cast<float*>(ws), L.err);
+                           static_cast<int>(mtiles), static_cast<int>(tiles),
+                           static_cast<int>(dp_tiles), early_weights ? 1 : 0,
+                           static_cast<float*>(ws), L.err);
     if (e != cudaSuccess) return e;
   }
-  if (!streamk || grid < 2) return cudaSuccess;
-  const SplitTiles st = split_tiles(tiles, KB, grid);
+  if (dp_tiles == tiles || grid < 2) return cudaSuccess;
+  SplitTiles st = split_tiles(tiles - dp_tiles, KB, grid);
   if (st.count == 0) return cudaSuccess;
-  const int mt = static_cast<int>(M < BT ? M : BT);
+  for (int i = 0; i < st.count; ++i) st.tile[i] += static_cast<int>(dp_tiles);
+  const int mt = static_cast<int>(M < TOK ? M : TOK);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(st.count), static_cast<unsigned>((mt + 7) / 8));
   cfg.blockDim = dim3(256);
@@ -708,8 +765,8 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, w8a16_streamk_fixup<BT>, st, static_cast<const float*>(ws), y,
-                            ldy, static_cast<int>(M), static_cast<int>(N));
+  return cudaLaunchKernelEx(&cfg, w8a16_streamk_fixup<TOK>, st, static_cast<const float*>(ws), y,
+                            ldy, static_cast<int>(M), static_cast<int>(N), static_cast<int>(mtiles));
 }
 
 }  // namespace
@@ -718,10 +775,17 @@ namespace {
 int token_tile(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
 }  // namespace
 
-// M <= 128 runs stream-K: FP32 partials of split tiles, two slots per CTA.
-size_t w8a16_workspace_bytes(int64_t M, int64_t, int64_t) {
-  if (M > 128) return 0;
-  return static_cast<size_t>(kStreamKMaxCtas) * 2 * token_tile(M) * 128 * sizeof(float);
+// M <= 128 runs stream-K: FP32 partials of split tiles, two slots per CTA
+// (required). M > 128 runs whole 256-token tiles and may run its last wave
+// stream-K: the same slots of [256][128] for up to 160 CTAs (optional).
+size_t w8a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 128) return streamk_bytes(kStreamKMaxCtas, token_tile(M));
+  const int64_t units = cdiv(M, 256) * cdiv(N, 128) * cdiv(K, 128);
+  return streamk_bytes(units < kStreamKMaxCtas ? units : kStreamKMaxCtas, 256);
+}
+
+size_t w8a16_workspace_required(int64_t M, int64_t N, int64_t K) {
+  return M <= 128 ? w8a16_workspace_bytes(M, N, K) : 0;
 }
 
 cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,

@@ -38,7 +38,11 @@ cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, c
                              uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                              bool after_act_quant);
 
+// Workspace of the W8A16 call: the size that enables every stream-K path,
+// and the part of it that is required (M <= 128; for M > 128 a smaller or
+// missing workspace runs every tile whole).
 size_t w8a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+size_t w8a16_workspace_required(int64_t M, int64_t N, int64_t K);
 // Always a programmatic dependent of the kernel before it; early_weights:
 // that kernel does not write q or scale_inv, so the weight stream may start
 // before it has completed (x, y and the workspace still wait for it).
@@ -57,6 +61,10 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
 
 // Sets the kernel's dynamic shared-memory limit once per device.
 cudaError_t ensure_smem_limit(const void* kernel, size_t bytes);
+
+// The workspace a linear call cannot run without (for W8A16 above 128 tokens
+// 0: its stream-K tail runs only when the workspace given is large enough).
+size_t required_workspace(int mode, int64_t M, int64_t N, int64_t K);
 
 // The launch context of the current device (checks compute capability 10.x).
 fp8blk_status current_launch(fp8blk_stream stream, Launch* L);

@@ -65,7 +65,7 @@ fp8blk_status fp8blk_streamed_linears(const fp8blk_linear_job* jobs, int64_t njo
     const float* s_dev = reinterpret_cast<const float*>(slot + round_up_sz(codes_bytes(j.N, j.ldq), kSlotAlign));
     const fp8blk_status st = validate_linear(j.x, j.ldx, slot, j.ldq, s_dev, j.y, j.ldy, j.M, j.N,
                                              j.K, workspace, workspace_bytes,
-                                             fp8blk_workspace_size(j.mode, j.M, j.N, j.K));
+                                             required_workspace(j.mode, j.M, j.N, j.K));
     if (st != FP8BLK_OK) return st;
   }
   Launch L;

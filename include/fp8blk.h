@@ -122,12 +122,18 @@ FP8BLK_EXPORT fp8blk_status fp8blk_quantize_act(const void* x, int64_t M, int64_
  *   x : BF16 [M][ldx], ldx >= K, ldx % 8 == 0                        (input)
  *   q : uint8 [N][ldq], ldq >= K, ldq % 16 == 0; scale_inv as above  (input)
  *   y : BF16 [M][ldy], ldy >= N, ldy % 8 == 0; must not alias the inputs (output)
- *   workspace : fp8blk_workspace_size(0, M, N, K) bytes, 256-byte aligned
- *               (may be NULL when that size is 0); its contents on entry do
- *               not matter and are scratch on return. For M <= 128 the slabs
- *               are split evenly over the SMs (stream-K) and the workspace
- *               holds the FP32 partials of tiles split between SMs (at most
- *               160 x 2 x 128 x 128 x 4 bytes); for M > 128 it is 0 bytes.
+ *   workspace : 256-byte aligned; its contents on entry do not matter and
+ *               are scratch on return.
+ *     - M <= 128: fp8blk_workspace_size(0, M, N, K) bytes are required. The
+ *       slabs are split evenly over the SMs (stream-K) and the workspace
+ *       holds the FP32 partials of tiles split between SMs (at most
+ *       160 x 2 x BT x 128 x 4 bytes, BT the token tile: 16, 32, 64 or 128).
+ *     - M > 128: optional. Tiles of 256 tokens run whole, one per SM at a
+ *       time; when the last wave of tiles would leave at least 15% of the SM
+ *       time idle and the workspace holds fp8blk_workspace_size(0, M, N, K)
+ *       bytes, that wave's slabs are split evenly over the SMs instead
+ *       (partials of [256][128] floats, two per SM). NULL or a smaller
+ *       workspace runs every tile whole.
  * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED_DEVICE, WORKSPACE, CUDA.
  * ------------------------------------------------------------------------- */
 FP8BLK_EXPORT fp8blk_status fp8blk_linear_w8a16(const void* x, int64_t ldx, const uint8_t* q, int64_t ldq,

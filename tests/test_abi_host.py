@@ -56,7 +56,10 @@ def test_workspace_size(lib):
     # W8A16: stream-K partials for M <= 128 (160 CTAs x 2 slots x BT x 128 floats)
     for m, bt in ((1, 16), (16, 16), (17, 32), (64, 64), (77, 128), (128, 128)):
         assert lib.fp8blk_workspace_size(0, m, N, K) == 160 * 2 * bt * 128 * 4
-    assert lib.fp8blk_workspace_size(0, 129, N, K) == 0
+    # M > 128 (optional, for the stream-K last wave): two [256][128] float
+    # slots per CTA, for min(160, tiles x KB) CTAs
+    assert lib.fp8blk_workspace_size(0, 129, N, K) == 2 * min(160, 1 * 8 * 8) * 256 * 128 * 4
+    assert lib.fp8blk_workspace_size(0, 512, 25600, 5120) == 2 * 160 * 256 * 128 * 4
     assert lib.fp8blk_workspace_size(1, M, N, 0) == 0
     assert lib.fp8blk_workspace_size(2, M, N, K) == 0
     assert lib.fp8blk_workspace_size(1, -1, N, K) == 0

@@ -317,6 +317,47 @@ def test_large_repeat_calls_are_deterministic(mode):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("M", [300, 512])
+def test_w8a16_stream_k_last_wave(M):
+    """Above 128 tokens the last wave of 256-token tiles runs stream-K when
+    the workspace allows (partials summed by the fix-up in slab order): the
+    output is within tolerance of the oracle on sampled rows, bit-identical
+    over repeated calls, and equal to the all-whole-tiles run (no
+    workspace) within the linear tolerance."""
+    wl = W.Workload(f"m{M}_k5120_n25600", M, 5120, 25600)
+    wb, q, s = weight_case(wl)
+    xb = synth.bf16_bits(wl.x_bf16())
+    x_d = to_dev_bf16(xb)
+    q_d, s_d = to_dev_u8(q), torch.from_numpy(s).to(DEV)
+    ws = torch.empty(fb.workspace_size(0, M, wl.N, wl.K), dtype=torch.uint8, device=DEV)
+    first = fb.linear_w8a16(x_d, q_d, s_d, workspace=ws)
+    out = torch.empty_like(first)
+    for _ in range(4):
+        fb.linear_w8a16(x_d, q_d, s_d, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), first.view(torch.int16))
+    rows = wl.checked_rows(64)
+    ref = oracle.linear_w8a16(xb, q, s, wl.N, wl.K, rows=rows)
+    check_linear(bf16_to_f64(first)[rows], ref, f"{wl.name}/stream-K last wave")
+    whole = bf16_to_f64(_w8a16_no_workspace(x_d, q_d, s_d))
+    check_linear(whole[rows], ref, f"{wl.name}/whole tiles")
+    assert fb.read_device_error() == 0
+
+
+def _w8a16_no_workspace(x, q, s):
+    """W8A16 through the C ABI with no workspace (every tile whole)."""
+    M, K = x.shape
+    N = q.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    st = fb.lib().fp8blk_linear_w8a16(x.data_ptr(), x.stride(0), q.data_ptr(), q.stride(0),
+                                      s.data_ptr(), y.data_ptr(), y.stride(0), M, N, K, None, 0,
+                                      torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("M", [1, 16, 64, 128])
 def test_small_m_repeat_calls_are_deterministic(M):
     """Stream-K at small token counts (both linears): split tiles are summed
