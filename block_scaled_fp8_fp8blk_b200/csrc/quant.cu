@@ -195,6 +195,10 @@ __global__ void __launch_bounds__(256, 2) quantize_weight_kernel(
   __shared__ uint32_t red[2][8];
   __shared__ int abort_flag;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // Launched as a programmatic dependent: the launch overlaps the kernel
+  // before, and nothing is read or written until that kernel has completed.
+  pdl_launch_dependents();
+  pdl_wait();
   if (tid == 0) {
     for (int s = 0; s < kCvtStages; ++s) mbar_init(&full[s], 1);
     mbar_init_fence();
@@ -316,6 +320,10 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
                                                          const float* __restrict__ scale_inv,
                                                          int64_t N, int64_t K, int KB,
                                                          uint16_t* __restrict__ w, int64_t ldw) {
+  // Launched as a programmatic dependent: the launch overlaps the kernel
+  // before, and nothing is read or written until that kernel has completed.
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * 8;
   for (int64_t n = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); n < N; n += warps) {
@@ -406,6 +414,23 @@ __global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ v
   }
 }
 
+// A launch as a programmatic dependent of the kernel before it in the stream.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 int grid_for_rows(int64_t rows, int num_sms) {
   const int64_t ctas = cdiv(rows, 8);
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
@@ -425,18 +450,16 @@ cudaError_t launch_quantize_weight(const Launch& L, const uint16_t* w, int64_t N
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(quantize_weight_kernel), kCvtSmem);
   if (e != cudaSuccess) return e;
   const int64_t nblocks = NB * KB, cap = 2 * static_cast<int64_t>(L.num_sms);
-  quantize_weight_kernel<<<static_cast<unsigned>(nblocks < cap ? nblocks : cap), 256, kCvtSmem,
-                           L.stream>>>(tw, N, K, q, ldq, scale_inv, static_cast<int>(KB),
-                                       static_cast<int>(nblocks), L.err);
-  return cudaGetLastError();
+  return launch_pdl(quantize_weight_kernel, static_cast<unsigned>(nblocks < cap ? nblocks : cap),
+                    256, kCvtSmem, L.stream, tw, N, K, q, ldq, scale_inv, static_cast<int>(KB),
+                    static_cast<int>(nblocks), L.err);
 }
 
 cudaError_t launch_dequantize(const Launch& L, const uint8_t* q, int64_t ldq,
                               const float* scale_inv, int64_t N, int64_t K, uint16_t* w,
                               int64_t ldw) {
-  dequantize_kernel<<<grid_for_rows(N, L.num_sms), 256, 0, L.stream>>>(
-      q, ldq, scale_inv, N, K, static_cast<int>(cdiv(K, 128)), w, ldw);
-  return cudaGetLastError();
+  return launch_pdl(dequantize_kernel, static_cast<unsigned>(grid_for_rows(N, L.num_sms)), 256, 0,
+                    L.stream, q, ldq, scale_inv, N, K, static_cast<int>(cdiv(K, 128)), w, ldw);
 }
 
 cudaError_t launch_quantize_act(const Launch& L, const uint16_t* x, int64_t M, int64_t K,
