@@ -381,8 +381,37 @@ def measure_targets(fb, dev, peaks, flush_l2, clock_sampler):
                                    "frac_measured": tf / pk, "frac_datasheet": tf / ds,
                                    "peak_measured": pk, "peak_datasheet": ds})
         del x, y, ws8
-    del q, s
     out["clocks_large_m"] = clock_sampler.stop()
+    # Sustained: W8A8 back to back for about a second per shape (the regime
+    # in which the sustained BF16 peak was measured: a seconds-long loop under
+    # the power cap), with its own clock record.
+    out["w8a8_sustained"] = []
+    for M in (4096, 16384):
+        x = activations(M, K)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws8 = torch.empty(max(1, fb.workspace_size(1, M, N, K)), dtype=torch.uint8, device=dev)
+        run = lambda: fb.linear_w8a8(x, q, s, out=y, workspace=ws8)
+        run()
+        torch.cuda.synchronize()
+        calls = max(20, int(1.0 / (out["large_m"][0 if M == 4096 else 2]["us"] * 1e-6)))
+        clock_sampler.start()
+        time.sleep(0.15)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(calls):
+            run()
+        b.record()
+        torch.cuda.synchronize()
+        clk = clock_sampler.stop()
+        us = 1e3 * a.elapsed_time(b) / calls
+        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        pk = FP8_OVER_BF16 * peaks["bf16_tflops_sustained"]
+        out["w8a8_sustained"].append({"M": M, "calls": calls, "us_per_call": us, "tflops": tf,
+                                      "peak_sustained": pk, "frac_sustained": tf / pk,
+                                      "frac_burst": tf / (FP8_OVER_BF16 * peaks["bf16_tflops"]),
+                                      "clocks": clk})
+        del x, y, ws8
+    del q, s
     torch.cuda.synchronize()
     assert fb.read_device_error() == 0
     w8a8_large = [r for r in out["large_m"] if r["mode"] == "w8a8"]
@@ -392,6 +421,8 @@ def measure_targets(fb, dev, peaks, flush_l2, clock_sampler):
                                                             for r in w8a16_small),
         "w8a8_m_ge_4096_min_frac_measured": min(r["frac_measured"] for r in w8a8_large),
         "w8a8_m_ge_4096_min_frac_datasheet": min(r["frac_datasheet"] for r in w8a8_large),
+        "w8a8_m_ge_4096_min_frac_sustained_back_to_back": min(r["frac_sustained"]
+                                                              for r in out["w8a8_sustained"]),
         "w8a8_target": 0.60,
         "w8a16_m_le_64_min_frac_measured": min(r["frac_measured"] for r in w8a16_small),
         "w8a16_m_le_64_min_frac_datasheet": min(r["frac_datasheet"] for r in w8a16_small),
