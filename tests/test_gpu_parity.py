@@ -124,6 +124,34 @@ def test_quantize_tie_heavy_blocks():
     assert np.array_equal(u8(q_d), q_ref)
 
 
+@pytest.mark.parametrize("amax_exp", [0, 120, -90])
+def test_quantize_every_mantissa_pair(amax_exp):
+    """One block per BF16 block-maximum mantissa (amax = 1.m x 2^amax_exp,
+    128 blocks) holding every BF16 mantissa at every exponent from the
+    maximum's down past the E4M3 zero threshold, both signs. E4M3(v / s)
+    depends on the two mantissas and the exponent gap only, so this covers
+    every case the converter's per-block multiplier (or, where none passes,
+    its product bracket) can meet at these magnitudes."""
+    blocks = []
+    for ma in range(128):
+        amax = (1.0 + ma / 128.0) * 2.0 ** amax_exp
+        vals = [amax]
+        for e in range(0, -26, -1):
+            v = (1.0 + np.arange(128) / 128.0) * 2.0 ** (amax_exp + e)
+            v = v[v <= amax]
+            vals.extend(np.stack([v, -v], axis=1).ravel().tolist())
+        blk = np.zeros(128 * 128, np.float64)
+        blk[:len(vals)] = vals
+        blocks.append(blk.reshape(128, 128))
+    w = np.concatenate(blocks, axis=1).astype(np.float32)
+    wb = synth.bf16_bits(synth.to_bf16(w))
+    assert np.array_equal((wb.astype(np.uint32) << 16).view(np.float32), w)  # exact in BF16
+    q_ref, s_ref = oracle.quantize_weight(wb)
+    q_d, s_d = fb.quantize_weight(to_dev_bf16(wb))
+    assert np.array_equal(s_d.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(u8(q_d), q_ref)
+
+
 def test_quantize_every_bf16_value():
     allb = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
     vals = (allb.astype(np.uint32) << 16).view(np.float32)
@@ -341,6 +369,35 @@ def test_w8a16_stream_k_last_wave(M):
     check_linear(bf16_to_f64(first)[rows], ref, f"{wl.name}/stream-K last wave")
     whole = bf16_to_f64(_w8a16_no_workspace(x_d, q_d, s_d))
     check_linear(whole[rows], ref, f"{wl.name}/whole tiles")
+    assert fb.read_device_error() == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode,N", [("w8a16", 384), ("w8a16", 1000), ("w8a8", 1000)])
+def test_large_token_raster_groups(mode, N):
+    """9000 tokens with K = 3000 put more activation bytes in flight than one
+    raster group holds, so the GEMMs walk their tiles in two unequal groups
+    (W8A16 with 256-token tiles: 18 + 18 of 36; W8A8 with 128-token tiles:
+    36 + 35 of 71). N = 384 leaves the W8A16 tiles in one short wave that
+    runs stream-K; N = 1000 is ragged. Sampled rows (spread over both groups)
+    match the oracle, and repeated calls are bit-identical."""
+    wl = W.Workload(f"m9000_k3000_n{N}", 9000, 3000, N)
+    wb, q, s = weight_case(wl)
+    xb = synth.bf16_bits(wl.x_bf16())
+    x_d = to_dev_bf16(xb)
+    q_d, s_d = to_dev_u8(q), torch.from_numpy(s).to(DEV)
+    f = fb.linear_w8a16 if mode == "w8a16" else fb.linear_w8a8
+    first = f(x_d, q_d, s_d)
+    again = f(x_d, q_d, s_d)
+    torch.cuda.synchronize()
+    assert torch.equal(again.view(torch.int16), first.view(torch.int16))
+    rows = np.unique(np.r_[wl.checked_rows(96), [0, 4607, 4608, 8999]])
+    if mode == "w8a16":
+        ref = oracle.linear_w8a16(xb, q, s, wl.N, wl.K, rows=rows)
+    else:
+        qx, sx = oracle.act_quant(xb)
+        ref = oracle.linear_w8a8(qx, sx, q, s, wl.N, wl.K, rows=rows)
+    check_linear(bf16_to_f64(first)[rows], ref, f"{mode}/{wl.name}")
     assert fb.read_device_error() == 0
 
 
