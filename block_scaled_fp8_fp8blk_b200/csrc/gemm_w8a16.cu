@@ -14,8 +14,10 @@
 // shared-memory write traffic.
 //
 // Persistent kernel: one CTA per SM walks tiles (NSUB x BT tokens by 128
-// weight rows; token tiles of one weight tile are neighbours in the order,
-// so they share it through L2), and every ring runs on across tiles. Each
+// weight rows) in raster groups (tile_coords: token tiles of one weight tile
+// are neighbours in the order, so they share it through L2, and a group of
+// token tiles, at most 48 MB of activations, meets every weight tile before
+// the next group starts), and every ring runs on across tiles. Each
 // sub-tile group ("item" i = NSUB * slab + t) is issued and committed by its
 // own MMA thread to a ring of "item done" barriers that every consumer reads
 // (the activation producer recycling slots, the expansion warps recycling A
@@ -219,11 +221,25 @@ __device__ __forceinline__ void expand_slabs(int eg, int total_slabs, const uint
   }
 }
 
-template <int BT, int NSUB>
+// Tile t -> (token tile, weight tile): in raster groups of gm token tiles
+// (GROUPED), else token tile t % mtiles of weight tile t / mtiles (one group;
+// the cheaper form keeps the epilogue within its registers).
+template <bool GROUPED>
+__device__ __forceinline__ void tile_of(int t, int mtiles, int ntiles_total, int gm, int& mt,
+                                        int& nt) {
+  if constexpr (GROUPED) {
+    tile_coords(t, mtiles, ntiles_total / mtiles, gm, mt, nt);
+  } else {
+    nt = t / mtiles;
+    mt = t % mtiles;
+  }
+}
+
+template <int BT, int NSUB, bool GROUPED>
 __global__ void __launch_bounds__(512, 1)
     w8a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_x,
                       const float* __restrict__ sw, __nv_bfloat16* __restrict__ y, int64_t ldy,
-                      int M, int N, int KB, int mtiles, int ntiles_total, int dp_tiles,
+                      int M, int N, int KB, int mtiles, int ntiles_total, int gm, int dp_tiles,
                       int early_weights, float* __restrict__ part, unsigned* __restrict__ err) {
   using C = W8A16Cfg<BT, NSUB>;
   extern __shared__ uint8_t smem_raw[];
@@ -287,7 +303,9 @@ __global__ void __launch_bounds__(512, 1)
       Schedule sc(KB, ntiles_total, dp_tiles);
       int tile, kb0, kb1;
       while (ok && sc.next(tile, kb0, kb1)) {
-        const int n0 = (tile / mtiles) * 128;
+        int mt, nt;
+        tile_of<GROUPED>(tile, mtiles, ntiles_total, gm, mt, nt);
+        const int n0 = nt * 128;
         for (int kb = kb0; kb < kb1; ++kb, ++j) {
           const int qs = j % C::QS;
           if (!mbar_wait_sleepy(&qempty[qs], ring_parity(j, C::QS) ^ 1u, err, kErrWaitLoad)) {
@@ -310,7 +328,9 @@ __global__ void __launch_bounds__(512, 1)
       Schedule sc(KB, ntiles_total, dp_tiles);
       int tile, kb0, kb1;
       while (ok && sc.next(tile, kb0, kb1)) {
-        const int m0 = (tile % mtiles) * (BT * NSUB);
+        int mt, nt;
+        tile_of<GROUPED>(tile, mtiles, ntiles_total, gm, mt, nt);
+        const int m0 = mt * (BT * NSUB);
         for (int kb = kb0; kb < kb1 && ok; ++kb) {
           for (int t = 0; t < NSUB; ++t, ++i) {
             const int xs = i % C::XS;
@@ -392,7 +412,9 @@ __global__ void __launch_bounds__(512, 1)
       Schedule sc(KB, ntiles_total, dp_tiles);
       int tile, kb0, kb1;
       while (ok && sc.next(tile, kb0, kb1)) {
-        const int m0 = (tile % mtiles) * (BT * NSUB), n0 = (tile / mtiles) * 128;
+        int mt, nt;
+        tile_of<GROUPED>(tile, mtiles, ntiles_total, gm, mt, nt);
+        const int m0 = mt * (BT * NSUB), n0 = nt * 128;
         const float* sw_row = sw + static_cast<int64_t>(n0 >> 7) * KB;
         uint64_t acc[64];  // acc[32t + p]: tokens 128t + 64h + 2p and 2p + 1
 #pragma unroll
@@ -488,7 +510,9 @@ __global__ void __launch_bounds__(512, 1)
       int tile, kb0, kb1;
       bool first_segment = true;
       while (ok && sc.next(tile, kb0, kb1)) {
-        const int m0 = (tile % mtiles) * (BT * NSUB), n0 = (tile / mtiles) * 128;
+        int tm, tn;
+        tile_of<GROUPED>(tile, mtiles, ntiles_total, gm, tm, tn);
+        const int m0 = tm * (BT * NSUB), n0 = tn * 128;
         const float* sw_row = sw + static_cast<int64_t>(n0 >> 7) * KB;
         uint64_t acc[BT / 2];
 #pragma unroll
@@ -634,15 +658,16 @@ template <int TOK>
 __global__ void __launch_bounds__(256) w8a16_streamk_fixup(const __grid_constant__ SplitTiles st,
                                                            const float* __restrict__ part,
                                                            uint16_t* __restrict__ y, int64_t ldy,
-                                                           int M, int N, int mtiles) {
+                                                           int M, int N, int mtiles, int gm) {
   pdl_launch_dependents();  // the next linear may be scheduled; it waits for this grid
   pdl_wait();
   const int i = static_cast<int>(blockIdx.x);
   const int r = threadIdx.x & 127;
-  const int t = st.tile[i];
-  const int n = (t / mtiles) * 128 + r;
+  int mt, nt;
+  tile_coords(st.tile[i], mtiles, (N + 127) / 128, gm, mt, nt);
+  const int n = nt * 128 + r;
   if (n >= N) return;
-  const int m0 = (t % mtiles) * TOK;
+  const int m0 = mt * TOK;
   const int c0 = st.c0[i], nc = st.ncontrib[i], slot0 = st.slot0[i];
   const int mbase = static_cast<int>(blockIdx.y) * 8 + (threadIdx.x >> 7);
   float acc[4];
@@ -673,7 +698,7 @@ size_t streamk_bytes(int64_t grid, int tok) {
   return static_cast<size_t>(grid) * 2 * tok * 128 * sizeof(float);
 }
 
-template <int BT, int NSUB>
+template <int BT, int NSUB, bool GROUPED>
 cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                       int64_t ldq, const float* sw, uint16_t* y, int64_t ldy, int64_t M,
                       int64_t N, int64_t K, void* ws, size_t ws_bytes, bool early_weights) {
@@ -684,7 +709,7 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, ldx * 2, 64, BT))
     return cudaErrorInvalidValue;
-  auto kern = w8a16_gemm_kernel<BT, NSUB>;
+  auto kern = w8a16_gemm_kernel<BT, NSUB, GROUPED>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
   {
@@ -700,6 +725,7 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
     if (regs != cudaSuccess) return regs;
   }
   const int64_t mtiles = cdiv(M, TOK), tiles = mtiles * cdiv(N, 128);
+  const int gm = GROUPED ? raster_group(mtiles, TOK * K * 2, kRasterBytesW8A16) : static_cast<int>(mtiles);
   // Slab and item counters are 32-bit per CTA.
   if (tiles * cdiv(K, 128) * NSUB > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   const int64_t KB = cdiv(K, 128);
@@ -745,7 +771,7 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, tq, tx, sw, reinterpret_cast<__nv_bfloat16*>(y), ldy,
                            static_cast<int>(M), static_cast<int>(N), static_cast<int>(KB),
-                           static_cast<int>(mtiles), static_cast<int>(tiles),
+                           static_cast<int>(mtiles), static_cast<int>(tiles), gm,
                            static_cast<int>(dp_tiles), early_weights ? 1 : 0,
                            static_cast<float*>(ws), L.err);
     if (e != cudaSuccess) return e;
@@ -766,7 +792,8 @@ cudaError_t launch_bt(const Launch& L, const uint16_t* x, int64_t ldx, const uin
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, w8a16_streamk_fixup<TOK>, st, static_cast<const float*>(ws), y,
-                            ldy, static_cast<int>(M), static_cast<int>(N), static_cast<int>(mtiles));
+                            ldy, static_cast<int>(M), static_cast<int>(N), static_cast<int>(mtiles),
+                            gm);
 }
 
 }  // namespace
@@ -791,11 +818,14 @@ size_t w8a16_workspace_required(int64_t M, int64_t N, int64_t K) {
 cudaError_t launch_w8a16_gemm(const Launch& L, const uint16_t* x, int64_t ldx, const uint8_t* q,
                               int64_t ldq, const float* sw, uint16_t* y, int64_t ldy, int64_t M,
                               int64_t N, int64_t K, void* ws, size_t ws_bytes, bool early_weights) {
-  if (M <= 16) return launch_bt<16, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
-  if (M <= 32) return launch_bt<32, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
-  if (M <= 64) return launch_bt<64, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
-  if (M <= 128) return launch_bt<128, 1>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
-  return launch_bt<128, 2>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  if (M <= 16) return launch_bt<16, 1, false>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  if (M <= 32) return launch_bt<32, 1, false>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  if (M <= 64) return launch_bt<64, 1, false>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  if (M <= 128) return launch_bt<128, 1, false>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  // Activations larger than the raster budget run in raster groups.
+  if (raster_group(cdiv(M, 256), 256 * K * 2, kRasterBytesW8A16) < cdiv(M, 256))
+    return launch_bt<128, 2, true>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
+  return launch_bt<128, 2, false>(L, x, ldx, q, ldq, sw, y, ldy, M, N, K, ws, ws_bytes, early_weights);
 }
 
 }  // namespace fp8blk

@@ -8,8 +8,10 @@
 // slab's FP32 partial ("promotion") rather than by the MMA.
 //
 // Persistent kernel: one CTA per SM walks output tiles of 128 tokens by 256
-// weight rows (two weight blocks), tile index t = m-tile + (#m-tiles) * n-tile
-// (token tiles of one weight tile are neighbours and share it through L2).
+// weight rows (two weight blocks) in raster groups (tile_coords): the token
+// tiles of one weight tile are neighbours and share it through L2, and a
+// group of token tiles (at most 24 MB of activation codes) meets every
+// weight tile before the next group starts.
 // Every ring runs on across tiles, so the next tile's loads and MMAs overlap
 // this tile's stores.
 //
@@ -88,7 +90,7 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
                      const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ sx,
                      int64_t ldsx, const float* __restrict__ sw, uint16_t* __restrict__ y,
                      int64_t ldy, int M, int N, int n_tma, int KB, int mtiles, int ntiles_total,
-                     int a_bytes, unsigned* __restrict__ err) {
+                     int gm, int a_bytes, unsigned* __restrict__ err) {
   using C = W8A8Cfg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_addr(smem_raw) & 1023u)) & 1023u;
@@ -101,6 +103,7 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles_n = ntiles_total / mtiles;
   const int my_tiles =
       static_cast<int>(blockIdx.x) < ntiles_total ? (ntiles_total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const int total_slabs = my_tiles * KB;
@@ -140,7 +143,9 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
       int j = 0;  // slab counter (across tiles)
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
-        const int row0 = is_a ? (tile % mtiles) * C::BM : (tile / mtiles) * C::BN;
+        int mt, nt;
+        tile_coords(tile, mtiles, ntiles_n, gm, mt, nt);
+        const int row0 = is_a ? mt * C::BM : nt * C::BN;
         for (int kb = 0; kb < KB; ++kb, ++j) {
           const int stage = j & (C::ST - 1);
           if (j >= C::ST) {  // the slab that last used this stage has finished
@@ -196,8 +201,10 @@ __global__ void __launch_bounds__(W8A8Cfg::THREADS, 1)
     int j = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles_total && ok; tile += gridDim.x) {
-      const int m0 = (tile % mtiles) * C::BM;
-      const int col0 = (tile / mtiles) * C::BN + 128 * h;  // first output column of this warp
+      int mt, nt;
+      tile_coords(tile, mtiles, ntiles_n, gm, mt, nt);
+      const int m0 = mt * C::BM;
+      const int col0 = nt * C::BN + 128 * h;  // first output column of this warp
       const bool has_cols = col0 < N;
       const int m = m0 + row;
       // sx is group-major with ldsx covering whole 128-row tiles, so rows
@@ -329,7 +336,8 @@ cudaError_t launch_w8a8_gemm(const Launch& L, const uint8_t* qx, int64_t ldqx, c
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, sx, ldsx, sw, y, ldy, static_cast<int>(M),
                             static_cast<int>(N), static_cast<int>(n_tma),
                             static_cast<int>(cdiv(K, 128)), static_cast<int>(mtiles),
-                            static_cast<int>(tiles), static_cast<int>(a_rows * 128), L.err);
+                            static_cast<int>(tiles), raster_group(mtiles, C::BM * K, kRasterBytesW8A8),
+                            static_cast<int>(a_rows * 128), L.err);
 }
 
 }  // namespace fp8blk

@@ -19,6 +19,19 @@ struct Launch {
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round_up(int64_t a, int64_t b) { return cdiv(a, b) * b; }
 
+// Token tiles per raster group of a persistent GEMM (see tile_coords): as
+// many as keep a group's activation rows within `budget` bytes, in groups of
+// near-equal size. Measured on the large-token linears: W8A8 with 24 MB of
+// activation codes per group; W8A16 with up to 48 MB of BF16 activations
+// (M = 4096 stays one group: two groups of 21 MB ran slower there).
+constexpr int64_t kRasterBytesW8A8 = 24ll << 20;
+constexpr int64_t kRasterBytesW8A16 = 48ll << 20;
+inline int raster_group(int64_t mtiles, int64_t bytes_per_mtile, int64_t budget) {
+  const int64_t most = bytes_per_mtile > 0 ? budget / bytes_per_mtile : mtiles;
+  const int64_t groups = cdiv(mtiles, most > 0 ? most : 1);
+  return static_cast<int>(cdiv(mtiles, groups > 0 ? groups : 1));
+}
+
 cudaError_t launch_quantize_weight(const Launch& L, const uint16_t* w, int64_t N, int64_t K,
                                    int64_t ldw, uint8_t* q, int64_t ldq, float* scale_inv);
 cudaError_t launch_dequantize(const Launch& L, const uint8_t* q, int64_t ldq,

@@ -498,4 +498,20 @@ __device__ __forceinline__ float bf16_hi_to_f32(uint32_t w) {
   return __uint_as_float(w & 0xFFFF0000u);
 }
 
+// Output tile t of a persistent GEMM -> (token tile, weight tile). Tiles run
+// in groups of gm token tiles: within a group the token tiles of one weight
+// tile are neighbours (they share its slabs through L2), and a group sweeps
+// every weight tile before the next group starts, so the group's activation
+// rows stay in L2 while the weight streams past. The last group may be
+// smaller.
+__device__ __forceinline__ void tile_coords(int t, int mtiles, int ntiles_n, int gm, int& mt,
+                                            int& nt) {
+  const int per = gm * ntiles_n;
+  const int first = (t / per) * gm;
+  const int r = t % per;
+  const int gsz = mtiles - first < gm ? mtiles - first : gm;
+  nt = r / gsz;
+  mt = first + r % gsz;
+}
+
 }  // namespace fp8blk
