@@ -381,6 +381,29 @@ def measure_targets(fb, dev, peaks, flush_l2, clock_sampler):
                                    "frac_measured": tf / pk, "frac_datasheet": tf / ds,
                                    "peak_measured": pk, "peak_datasheet": ds})
         del x, y, ws8
+    # A library FP8 GEMM on the same shapes and on 8192^3 (torch._scaled_mm:
+    # E4M3 operands, one FP32 scale per tensor, BF16 out, timed like the
+    # calls above): this box's measured FP8 tensor rate for a GEMM without
+    # block scales, next to the W8A8 linears.
+    out["library_fp8"] = []
+    try:
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        for M, Kl, Nl in ((4096, K, N), (16384, K, N), (8192, 8192, 8192)):
+            a8 = torch.randn(M, Kl, device=dev, generator=g).to(torch.float8_e4m3fn)
+            b8 = torch.randn(Nl, Kl, device=dev, generator=g).to(torch.float8_e4m3fn)
+            us = timed(lambda: torch._scaled_mm(a8, b8.t(), scale_a=one, scale_b=one,
+                                                out_dtype=torch.bfloat16), 5 if M > 8192 else 10)
+            tf = 2.0 * M * Nl * Kl / (us * 1e-6) / 1e12
+            rec = {"M": M, "K": Kl, "N": Nl, "us": us, "tflops": tf,
+                   "frac_of_2x_bf16_burst": tf / (FP8_OVER_BF16 * peaks["bf16_tflops"])}
+            ours = [r for r in out["large_m"] if r["mode"] == "w8a8" and r["M"] == M
+                    and (Kl, Nl) == (K, N)]
+            if ours:
+                rec["w8a8_linear_over_library"] = ours[0]["tflops"] / tf
+            out["library_fp8"].append(rec)
+            del a8, b8
+    except (RuntimeError, TypeError) as e:
+        out["library_fp8"] = {"unavailable": str(e).splitlines()[0][:200]}
     out["clocks_large_m"] = clock_sampler.stop()
     # Sustained: W8A8 back to back for about a second per shape (the regime
     # in which the sustained BF16 peak was measured: a seconds-long loop under
