@@ -414,56 +414,126 @@ __global__ void __launch_bounds__(256, 2) quantize_weight_kernel(
 }
 
 // ----------------------------------------------------------- dequantizer
-// w[n][k] = BF16(float(E4M3(q[n][k])) * s[n/128][k/128]): one warp per row at
-// a time, 16 codes (one 16-byte load, two 16-byte stores) per lane-step.
+// w[n][k] = BF16(float(E4M3(q[n][k])) * s[n/128][k/128]), one float multiply
+// and one round to nearest even. Persistent, one CTA of 512 threads per SM,
+// over tiles of 64 rows x 256 codes (tile t: row tile t / tiles_k, column
+// tile t % tiles_k). Thread 0 keeps a 4-stage ring of TMA loads of code
+// tiles (16 KB, unswizzled; parts past N or K read as 0) and TMA-stores each
+// finished BF16 tile (32 KB, three staging buffers; the store clips at N and
+// K), so the bytes in flight sit in shared memory, not in registers. Every
+// thread converts two 16-code chunks per tile (chunk c = thread + 512 u:
+// row c / 16, codes 16 (c % 16) ...), reading the stage conflict-free and
+// writing its 32 bytes of BF16 in the half order that keeps a quarter warp
+// on distinct banks. A tile's two block scales are loaded during the tile
+// before.
 __device__ __forceinline__ uint32_t dequant2(uint32_t codes16, float s) {
   const uint32_t h2 = e4m3x2_to_f16x2(codes16);
   return cvt_bf16x2(__fmul_rn(f16_hi_to_f32(h2), s), __fmul_rn(f16_lo_to_f32(h2), s));
 }
 
-__global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ q, int64_t ldq,
-                                                         const float* __restrict__ scale_inv,
-                                                         int64_t N, int64_t K, int KB,
-                                                         uint16_t* __restrict__ w, int64_t ldw) {
+constexpr int kDqRows = 64, kDqCols = 256;
+constexpr int kDqInBytes = kDqRows * kDqCols;       // one code tile
+constexpr int kDqOutBytes = kDqRows * kDqCols * 2;  // its BF16 tile
+constexpr int kDqStages = 4, kDqOutBufs = 3, kDqThreads = 512;
+constexpr size_t kDqSmem = 128 + static_cast<size_t>(kDqStages) * kDqInBytes +
+                           static_cast<size_t>(kDqOutBufs) * kDqOutBytes;
+
+__global__ void __launch_bounds__(kDqThreads, 1) dequantize_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_w,
+    const float* __restrict__ scale_inv, int KB, int tiles_k, int ntiles, unsigned* __restrict__ err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
+  uint8_t* s_in = smem;                                 // kDqStages code tiles
+  uint8_t* s_out = smem + kDqStages * kDqInBytes;       // kDqOutBufs BF16 tiles
+  __shared__ uint64_t full[kDqStages];
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x;
   // Launched as a programmatic dependent: the launch overlaps the kernel
   // before, and nothing is read or written until that kernel has completed.
   pdl_launch_dependents();
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * 8;
-  for (int64_t n = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); n < N; n += warps) {
-    const uint8_t* qrow = q + n * ldq;
-    uint16_t* wrow = w + n * ldw;
-    const float* srow = scale_inv + (n >> 7) * KB;
-    // Four 16-code chunks per lane per step: all four loads are issued before
-    // any conversion, so each warp keeps 2 KB of reads in flight.
-    for (int64_t base = 0; base < K; base += 4 * 32 * 16) {
-      uint4 c[4];
-      float s[4];
+  if (tid == 0) {
+    for (int st = 0; st < kDqStages; ++st) mbar_init(&full[st], 1);
+    mbar_init_fence();
+    abort_flag = 0;
+  }
+  __syncthreads();
+  // Thread 0: load this CTA's i-th tile into stage i % kDqStages.
+  auto issue = [&](int i) {
+    const int t = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    if (t >= ntiles) return;
+    const int tr = t / tiles_k, tc = t - tr * tiles_k;
+    uint64_t* bar = &full[i % kDqStages];
+    mbar_arrive_expect_tx(bar, kDqInBytes);
+    tma_load_2d(s_in + (i % kDqStages) * kDqInBytes, &tm_q, bar, tc * kDqCols, tr * kDqRows);
+  };
+  if (tid == 0) {
+    tma_prefetch_map(&tm_q);
+    tma_prefetch_map(&tm_w);
+    for (int i = 0; i < kDqStages; ++i) issue(i);
+  }
+  const int h = (tid >> 2) & 1;  // which 16-byte half of its 32 output bytes a thread writes first
+  // The block scales of this CTA's i-th tile (0 past K).
+  auto scales = [&](int i, float& s0, float& s1) {
+    const int t = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    s0 = s1 = 0.0f;
+    if (t >= ntiles) return;
+    const int tr = t / tiles_k, tc = t - tr * tiles_k;
+    const float* srow = scale_inv + static_cast<int64_t>((tr * kDqRows) >> 7) * KB;
+    const int kb0 = tc * (kDqCols / 128);
+    if (kb0 < KB) s0 = __ldg(srow + kb0);
+    if (kb0 + 1 < KB) s1 = __ldg(srow + kb0 + 1);
+  };
+  float s0, s1;
+  scales(0, s0, s1);
+  int i = 0;
+  for (;; ++i) {
+    const int t = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    if (t >= ntiles) break;
+    const int st = i % kDqStages;
+    const bool landed = mbar_wait_warp(&full[st], static_cast<uint32_t>((i / kDqStages) & 1), err,
+                                       kErrWaitLoad);
+    if (tid == 0) tma_store_wait_read<kDqOutBufs - 1>();  // the store that last used this buffer has read it
+    if ((tid & 31) == 0 && !landed) abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) break;
+    float n0, n1;
+    scales(i + 1, n0, n1);
+    const int tr = t / tiles_k, tc = t - tr * tiles_k;
+    const uint8_t* in = s_in + st * kDqInBytes;
+    uint8_t* out = s_out + (i % kDqOutBufs) * kDqOutBytes;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t k = base + u * 512 + lane * 16;
-        c[u] = make_uint4(0, 0, 0, 0);
-        s[u] = 0.0f;
-        if (k < K) s[u] = __ldg(srow + (k >> 7));
-        if (k + 16 <= K) c[u] = __ldcs(reinterpret_cast<const uint4*>(qrow + k));
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t k = base + u * 512 + lane * 16;
-        if (k + 16 <= K) {
-          const uint4 o0 = make_uint4(dequant2(c[u].x, s[u]), dequant2(c[u].x >> 16, s[u]),
-                                      dequant2(c[u].y, s[u]), dequant2(c[u].y >> 16, s[u]));
-          const uint4 o1 = make_uint4(dequant2(c[u].z, s[u]), dequant2(c[u].z >> 16, s[u]),
-                                      dequant2(c[u].w, s[u]), dequant2(c[u].w >> 16, s[u]));
-          __stcs(reinterpret_cast<uint4*>(wrow + k), o0);
-          __stcs(reinterpret_cast<uint4*>(wrow + k + 8), o1);
-        } else if (k < K) {
-          for (int64_t t = k; t < K; ++t)
-            wrow[t] = static_cast<uint16_t>(dequant2(qrow[t], s[u]) & 0xFFFFu);
-        }
+    for (int u = 0; u < kDqInBytes / 16 / kDqThreads; ++u) {
+      const int c = tid + kDqThreads * u;
+      const uint4 v = *reinterpret_cast<const uint4*>(in + 16 * c);
+      const float sc = (c & 15) < 8 ? s0 : s1;
+      const uint4 o0 = make_uint4(dequant2(v.x, sc), dequant2(v.x >> 16, sc), dequant2(v.y, sc),
+                                  dequant2(v.y >> 16, sc));
+      const uint4 o1 = make_uint4(dequant2(v.z, sc), dequant2(v.z >> 16, sc), dequant2(v.w, sc),
+                                  dequant2(v.w >> 16, sc));
+      uint8_t* dst = out + (c >> 4) * (2 * kDqCols) + (c & 15) * 32;
+      *reinterpret_cast<uint4*>(dst + 16 * h) = h ? o1 : o0;
+      *reinterpret_cast<uint4*>(dst + 16 * (1 - h)) = h ? o0 : o1;
+    }
+    s0 = n0;
+    s1 = n1;
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tma_store_2d(&tm_w, out, tc * kDqCols, tr * kDqRows);
+      tma_store_commit();
+      issue(i + kDqStages);  // every thread is done with stage st
+    }
+  }
+  if (tid == 0) {
+    // After a time-out, the loads still in flight land before the CTA exits.
+    if (abort_flag) {
+      for (int k = i; k < i + kDqStages; ++k) {
+        const int t = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+        if (t < ntiles) mbar_wait(&full[k % kDqStages], static_cast<uint32_t>((k / kDqStages) & 1), err, kErrWaitLoad);
       }
     }
+    tma_store_wait_all();
   }
 }
 
@@ -536,12 +606,6 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, 
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-int grid_for_rows(int64_t rows, int num_sms) {
-  const int64_t ctas = cdiv(rows, 8);
-  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
-  return static_cast<int>(ctas < cap ? ctas : cap);
-}
-
 }  // namespace
 
 cudaError_t launch_quantize_weight(const Launch& L, const uint16_t* w, int64_t N, int64_t K,
@@ -563,8 +627,20 @@ cudaError_t launch_quantize_weight(const Launch& L, const uint16_t* w, int64_t N
 cudaError_t launch_dequantize(const Launch& L, const uint8_t* q, int64_t ldq,
                               const float* scale_inv, int64_t N, int64_t K, uint16_t* w,
                               int64_t ldw) {
-  return launch_pdl(dequantize_kernel, static_cast<unsigned>(grid_for_rows(N, L.num_sms)), 256, 0,
-                    L.stream, q, ldq, scale_inv, N, K, static_cast<int>(cdiv(K, 128)), w, ldw);
+  const int64_t tiles_k = cdiv(K, kDqCols), ntiles = cdiv(N, kDqRows) * tiles_k;
+  if (ntiles > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  CUtensorMap tq, tw;
+  if (!make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K, N, ldq, kDqCols, kDqRows,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, K, N, 2 * ldw, kDqCols, kDqRows,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dequantize_kernel), kDqSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = ntiles < L.num_sms ? ntiles : L.num_sms;
+  return launch_pdl(dequantize_kernel, static_cast<unsigned>(grid), kDqThreads, kDqSmem, L.stream, tq, tw,
+                    scale_inv, static_cast<int>(cdiv(K, 128)), static_cast<int>(tiles_k),
+                    static_cast<int>(ntiles), L.err);
 }
 
 cudaError_t launch_quantize_act(const Launch& L, const uint16_t* x, int64_t M, int64_t K,
