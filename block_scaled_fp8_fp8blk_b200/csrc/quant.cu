@@ -424,8 +424,7 @@ __global__ void __launch_bounds__(256, 2) quantize_weight_kernel(
 // thread converts two 16-code chunks per tile (chunk c = thread + 512 u:
 // row c / 16, codes 16 (c % 16) ...), reading the stage conflict-free and
 // writing its 32 bytes of BF16 in the half order that keeps a quarter warp
-// on distinct banks. A tile's two block scales are loaded during the tile
-// before.
+// on distinct banks. A tile's two block scales are loaded two tiles ahead.
 __device__ __forceinline__ uint32_t dequant2(uint32_t codes16, float s) {
   const uint32_t h2 = e4m3x2_to_f16x2(codes16);
   return cvt_bf16x2(__fmul_rn(f16_hi_to_f32(h2), s), __fmul_rn(f16_lo_to_f32(h2), s));
@@ -484,8 +483,9 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequantize_kernel(
     if (kb0 < KB) s0 = __ldg(srow + kb0);
     if (kb0 + 1 < KB) s1 = __ldg(srow + kb0 + 1);
   };
-  float s0, s1;
+  float s0, s1, n0, n1;
   scales(0, s0, s1);
+  scales(1, n0, n1);
   int i = 0;
   for (;; ++i) {
     const int t = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
@@ -497,8 +497,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequantize_kernel(
     if ((tid & 31) == 0 && !landed) abort_flag = 1;
     __syncthreads();
     if (abort_flag) break;
-    float n0, n1;
-    scales(i + 1, n0, n1);
+    float p0, p1;
+    scales(i + 2, p0, p1);
     const int tr = t / tiles_k, tc = t - tr * tiles_k;
     const uint8_t* in = s_in + st * kDqInBytes;
     uint8_t* out = s_out + (i % kDqOutBufs) * kDqOutBytes;
@@ -517,6 +517,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequantize_kernel(
     }
     s0 = n0;
     s1 = n1;
+    n0 = p0;
+    n1 = p1;
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
