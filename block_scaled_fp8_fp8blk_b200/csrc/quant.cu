@@ -1,8 +1,9 @@
 // Elementwise stages of the block-FP8 linear: the weight converter, the
 // dequantizer, the 1 x 128 activation quantizer and the bare E4M3 codec.
-// All are HBM-bound streams: 16-byte vector loads and stores, one pass over
-// the data (the converter keeps its 128 x 128 block in registers between the
-// amax reduction and the encoding).
+// All are HBM-bound streams with one pass over the data: the converter and
+// the dequantizer move tiles with TMA (the converter keeps its 128 x 128
+// block in registers between the amax reduction and the encoding), the
+// activation quantizer and the codec use 16-byte vector loads and stores.
 #include "internal.cuh"
 #include "ptx.cuh"
 
