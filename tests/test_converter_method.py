@@ -9,6 +9,7 @@ block that takes a multiplier. The codes are the converter's definition
 (FastVideo PR #1829, "Changes", converter bullet: W / s with s = amax / 448,
 rounded to E4M3); the GPU tests then compare the kernel with the oracle."""
 import os
+import platform
 import shutil
 import subprocess
 
@@ -20,7 +21,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
 def test_multiplier_gives_the_quotient_codes_for_every_bf16_pair(tmp_path):
     exe = tmp_path / "check"
-    subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-msse2", "-mfpmath=sse", "-o", str(exe),
+    # IEEE single precision with round to nearest and no fused multiply-add
+    # (x86 would otherwise be free to use x87 extended precision)
+    x86 = platform.machine().lower() in ("x86_64", "amd64", "i686", "i386")
+    flags = ["-O2", "-ffp-contract=off"] + (["-msse2", "-mfpmath=sse"] if x86 else [])
+    subprocess.run(["gcc", *flags, "-o", str(exe),
                     os.path.join(HERE, "native", "converter_multiplier_check.c"), "-lm",
                     "-lpthread"], check=True)
     threads = max(1, min(32, os.cpu_count() or 1))
