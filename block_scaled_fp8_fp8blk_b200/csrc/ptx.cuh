@@ -504,8 +504,8 @@ __device__ __forceinline__ float bf16_hi_to_f32(uint32_t w) {
 // every weight tile before the next group starts, so the group's activation
 // rows stay in L2 while the weight streams past. The last group may be
 // smaller.
-__device__ __forceinline__ void tile_coords(int t, int mtiles, int ntiles_n, int gm, int& mt,
-                                            int& nt) {
+__host__ __device__ __forceinline__ void tile_coords(int t, int mtiles, int ntiles_n, int gm,
+                                                     int& mt, int& nt) {
   const int per = gm * ntiles_n;
   const int first = (t / per) * gm;
   const int r = t % per;
