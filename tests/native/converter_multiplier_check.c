@@ -1,4 +1,4 @@
-// Exhaustive CPU check of the converter's per-block multiplier (test code).
+// Exhaustive CPU check of the converter's two encoders (test code).
 //
 // The GPU converter encodes a 128 x 128 block with divisor d = RN(amax / 448)
 // as E4M3(RN(v * c)) for a multiplier c that it first checks on the 128 BF16
@@ -9,7 +9,12 @@
 // selection in FP32 (SSE, round to nearest even, no contraction) for every
 // positive finite BF16 block maximum, and for each block with a passing c
 // compares E4M3(RN(v * c)) with E4M3(RN(v / d)) for every BF16 v with
-// |v| <= amax, both signs. It prints the counts and exits 1 on any mismatch.
+// |v| <= amax, both signs. It also checks the converter's other encoder,
+// the product bracket, for every block with d >= 2^-125: with y = RN(1/d),
+// ylo = RN(y (1 - 2^-21)) and yhi = RN(y (1 + 2^-21)), whenever the codes of
+// RN(v * ylo) and RN(v * yhi) agree they must equal the quotient's code (the
+// other elements, the straddles, are divided exactly). It prints the counts
+// and exits 1 on any mismatch.
 // The E4M3 rounding here is its own: the nearest of the 127 finite
 // magnitudes, ties to the even code, saturating at 448.
 #include <math.h>
@@ -62,13 +67,34 @@ static int passes(float d, float c) {
 typedef struct {
   int t, nt;
   long long blocks, chosen[3], none, pairs, bad;
+  long long bracket_pairs, straddles, bracket_bad;
 } Job;
+
+// The bracket over every BF16 v of the block with maximum bits ab (d >= 2^-125).
+static void bracket(Job* J, uint32_t ab, float d) {
+  volatile float y = 1.0f / d;
+  volatile float ylo = y * 0.99999952316284180f;  // 1 - 2^-21
+  volatile float yhi = y * 1.00000047683715820f;  // 1 + 2^-21
+  for (uint32_t vb = 0; vb <= ab; ++vb)
+    for (int sg = 0; sg < 2; ++sg) {
+      volatile float v = f_of((vb | (sg ? 0x8000u : 0u)) << 16);
+      volatile float plo = v * ylo, phi = v * yhi, q = v / d;
+      const uint8_t clo = e4m3(plo), chi = e4m3(phi);
+      ++J->bracket_pairs;
+      if (clo != chi) { ++J->straddles; continue; }
+      if (clo != e4m3(q)) {
+        if (J->bracket_bad < 5) printf("bracket mismatch: amax bits %04x, v bits %04x\n", ab, vb);
+        ++J->bracket_bad;
+      }
+    }
+}
 
 static void* run(void* arg) {
   Job* J = (Job*)arg;
   for (uint32_t ab = 1 + (uint32_t)J->t; ab < 0x7F80u; ab += (uint32_t)J->nt) {
     volatile float amax = f_of(ab << 16);
     volatile float d = amax / 448.0f;
+    if (d >= 2.35098870e-38f) bracket(J, ab, d);  // 2^-125: the bracket's range
     if (d < 7.88860905e-31f) continue;  // 2^-100: not a multiplier block
     ++J->blocks;
     volatile float c0 = 1.0f / d;
@@ -105,6 +131,7 @@ int main(int argc, char** argv) {
     pthread_create(&th[t], NULL, run, &job[t]);
   }
   long long blocks = 0, chosen[3] = {0, 0, 0}, none = 0, pairs = 0, bad = 0;
+  long long bpairs = 0, straddles = 0, bbad = 0;
   for (int t = 0; t < nt; ++t) {
     pthread_join(th[t], NULL);
     blocks += job[t].blocks;
@@ -112,8 +139,12 @@ int main(int argc, char** argv) {
     none += job[t].none;
     pairs += job[t].pairs;
     bad += job[t].bad;
+    bpairs += job[t].bracket_pairs;
+    straddles += job[t].straddles;
+    bbad += job[t].bracket_bad;
   }
-  printf("blocks %lld rn %lld up %lld down %lld none %lld pairs %lld mismatches %lld\n", blocks,
-         chosen[0], chosen[1], chosen[2], none, pairs, bad);
-  return bad != 0;
+  printf("blocks %lld rn %lld up %lld down %lld none %lld pairs %lld mismatches %lld "
+         "bracket_pairs %lld straddles %lld bracket_mismatches %lld\n",
+         blocks, chosen[0], chosen[1], chosen[2], none, pairs, bad, bpairs, straddles, bbad);
+  return bad != 0 || bbad != 0;
 }

@@ -1,5 +1,6 @@
-"""The converter's per-block multiplier, checked on the CPU over its whole
-domain (every BF16 block maximum x every BF16 value; about 10^9 pairs).
+"""The converter's two encoders, checked on the CPU over their whole domain
+(every BF16 block maximum x every BF16 value; about 10^9 pairs each): the
+per-block multiplier and the product bracket it falls back to.
 
 The GPU converter (csrc/quant.cu, verify_multiplier) encodes a block with
 one multiply per element by a multiplier c it has checked on the 128 BF16
@@ -33,6 +34,9 @@ def test_multiplier_gives_the_quotient_codes_for_every_bf16_pair(tmp_path):
     line = out.stdout.strip().splitlines()[-1]
     f = dict(zip(line.split()[0::2], (int(v) for v in line.split()[1::2])))
     assert out.returncode == 0 and f["mismatches"] == 0, out.stdout
+    # the product bracket: equal ends always give the quotient's code
+    assert f["bracket_mismatches"] == 0 and f["bracket_pairs"] > 1.0e9, out.stdout
+    assert 0 < f["straddles"] < 0.05 * f["bracket_pairs"]
     # every usable block maximum was tried, about 10^9 pairs compared
     assert f["blocks"] == 28064 and f["pairs"] > 9.8e8
     # most blocks take the multiplier (the rest keep the product bracket)
